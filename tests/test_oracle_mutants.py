@@ -1,0 +1,46 @@
+"""Plant plausible mistakes in a copy of the oracle and check the pins catch them.
+
+Each mutant is one textual change to oracle/dg_oracle.c, compiled on the CPU
+into a temporary library; the pin suite (tests/test_oracle_pins.py) is then
+run against it in a subprocess and must fail.  The real oracle is untouched.
+"""
+import os
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+SRC = os.path.join(ROOT, "oracle", "dg_oracle.c")
+
+MUTANTS = {
+    "sb_index_transposed": ("sb[(int64_t)nb * nkb + kb]", "sb[(int64_t)kb * nkb + nb]"),
+    "sb_block_ignored": ("int nb = n / 128;", "int nb = 0;"),
+    "k_tail_dropped": ("int k1 = k0 + 128 < K ? k0 + 128 : K;", "int k1 = k0 + 128 < K ? k0 + 128 : k0;"),
+    "b_transposed": ("double t = g_e4m3[a[k]] * g_e4m3[bn[k]];",
+                     "double t = g_e4m3[a[k]] * g_e4m3[b[(int64_t)k * N + n]];"),
+    "bf16_truncates": ("if (frac > 0.5)", "if (frac > 2.0)"),
+    "e4m3_bias_8": ("v = ldexp(1.0 + (double)m / 8.0, e - 7);", "v = ldexp(1.0 + (double)m / 8.0, e - 8);"),
+    "sa_not_transposed": ("sa_m[(int64_t)kb * sa_stride]", "sa_m[kb]"),
+    "products_lose_sign": ("p += t;", "p += fabs(t);"),
+    "contiguous_ignores_group": ("B + (int64_t)g * N * K, sb + (int64_t)g * nbn * nkb, N, K,\n                 D + m * N",
+                                 "B, sb, N, K,\n                 D + m * N"),
+    "masked_off_by_one": ("if (m >= masked_m[g]) continue;", "if (m > masked_m[g]) continue;"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_pins_reject_mutant(name, tmp_path):
+    old, new = MUTANTS[name]
+    src = open(SRC).read()
+    assert src.count(old) == 1, f"mutation site for {name} not found exactly once"
+    mut = tmp_path / "mutant.c"
+    mut.write_text(src.replace(old, new))
+    so = tmp_path / "libmutant.so"
+    subprocess.run(["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c11", "-ffp-contract=off",
+                    str(mut), "-o", str(so), "-lm"], check=True)
+    env = dict(os.environ, DG_ORACLE_SO=str(so), OMP_NUM_THREADS="2")
+    r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
+                        os.path.join(ROOT, "tests", "test_oracle_pins.py")],
+                       cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
+    assert r.returncode != 0, f"mutant {name} passed every pin:\n{r.stdout[-2000:]}"
