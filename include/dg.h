@@ -1,0 +1,160 @@
+/*
+ * dg.h -- C ABI of the B200 (sm_100a) FP8 block-scaled NT GEMM library.
+ *
+ * Operation (page "DeepGEMM项目介绍与本地部署指南" -- DeepGEMM project
+ * introduction and local deployment guide -- section "接口" (Interface); scale
+ * granularity and the 128-wide promotion interval from the page "Deepseek
+ * DeepGEMM 技术原理的深入分析", section "技术背景与核心原理"):
+ *
+ *   D[m,n] = bf16( sum_kb sa[m,kb] * sb[n/128,kb] * sum_{k in block kb} A[m,k]*B[n,k] )
+ *
+ * with A, B in FP8 e4m3 (OCP E4M3FN), FP32 scales per 1x128 row tile of A (sa)
+ * and per 128x128 block of B (sb), FP32 accumulation in which every 128-wide
+ * K block's partial product is scaled and added separately, and a bf16 result
+ * rounded to nearest even.
+ *
+ * Common conventions for every entry point below
+ * ----------------------------------------------
+ *  Pointers   All tensor pointers are CUDA DEVICE pointers, 16-byte aligned,
+ *             owned by the caller.  The library never allocates, frees or
+ *             keeps them past the call.
+ *  Layouts    A   uint8 (e4m3 codes) [rows][K], K contiguous.
+ *             B   uint8 (e4m3 codes) [G][N][K], K contiguous ("NT": the RHS is
+ *                 stored transposed).  G = 1 for the dense call.
+ *             sa  float32, TRANSPOSED: element (m, kb) at sa[kb*sa_stride + m]
+ *                 (masked: group g's block starts at g*ceil(K/128)*sa_stride).
+ *                 sa_stride >= rows and a multiple of 4 (16 bytes), e.g.
+ *                 dg_get_tma_aligned_size(rows, 4).
+ *             sb  float32 [G][ceil(N/128)][ceil(K/128)], row-major.
+ *             D   bf16 bits (uint16) [rows][N] row-major (masked: [G][M_max][N]).
+ *  Limits     K % 128 == 0, N % 8 == 0 (16-byte rows of D), K and N >= 1.
+ *  Stream     `stream` is a cudaStream_t (NULL = legacy default stream).  The
+ *             call only enqueues work: it does not synchronise, read device
+ *             memory from the host, or allocate, so it may be captured in a
+ *             CUDA graph.
+ *  Errors     Bad arguments are reported synchronously as a dg_status and
+ *             nothing is launched (dg_last_error_message() says why).  A
+ *             launch failure returns DG_ERR_CUDA.  Bad DEVICE-side data
+ *             (m_indices outside [-1,G), masked_m outside [0,M_max]) cannot be
+ *             seen by the host: the kernel skips the offending rows/groups
+ *             (masked_m is clamped) and sets a bit in the device error word,
+ *             read with dg_get_device_error().  Every wait inside the kernels
+ *             is bounded; a wait that runs out sets DG_DEVERR_TIMEOUT and the
+ *             kernel returns instead of hanging.
+ *  Threads    dg_set_num_sms() is process-global; all other calls are
+ *             reentrant.
+ */
+#ifndef DG_H_
+#define DG_H_
+
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define DG_API __attribute__((visibility("default")))
+#else
+#define DG_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum dg_status {
+    DG_OK = 0,
+    DG_ERR_INVALID_ARG = 1,  /* null pointer, non-positive size, bad stride     */
+    DG_ERR_UNSUPPORTED = 2,  /* valid in the math but not on this path (K%128)  */
+    DG_ERR_MISALIGNED = 3,   /* a pointer is not 16-byte aligned                */
+    DG_ERR_CUDA = 4          /* a CUDA runtime/driver call or launch failed     */
+} dg_status;
+
+/* Bits of the device error word (dg_get_device_error). */
+#define DG_DEVERR_TIMEOUT 1u        /* a bounded wait inside a kernel ran out  */
+#define DG_DEVERR_BAD_M_INDEX 2u    /* contiguous: m_indices value not in [-1,G) */
+#define DG_DEVERR_BAD_MASKED_M 4u   /* masked: masked_m value not in [0,M_max]  */
+
+/*
+ * Dense GEMM: D[M,N] = scaled A[M,K] . B[N,K]^T (section "常规密集型 GEMM（非分组）",
+ * the non-grouped call of the Interface section).
+ *   D          uint16 bf16 [M][N]
+ *   A          uint8 e4m3 [M][K]
+ *   sa         float32 transposed, sa[kb*sa_stride + m], kb < K/128
+ *   B          uint8 e4m3 [N][K]
+ *   sb         float32 [ceil(N/128)][K/128]
+ * M == 0 is a valid empty problem (returns DG_OK, launches nothing).
+ */
+DG_API dg_status dg_fp8_gemm_nt(uint16_t* D, const uint8_t* A, const float* sa, int sa_stride,
+                         const uint8_t* B, const float* sb, int M, int N, int K, void* stream);
+
+/*
+ * Grouped GEMM, contiguous layout (section "分组 GEMM（连续布局）"): the rows of
+ * all groups are concatenated along M and share N and K.  m_indices[m] (int32,
+ * device) is the group of row m; -1 marks a padding row, whose D row is left
+ * untouched.  Each group's segment must start on a multiple of
+ * dg_get_m_alignment_for_contiguous_layout() rows, so M_total is a multiple
+ * of it.  Row m uses B + g*N*K and sb + g*ceil(N/128)*(K/128).
+ *   D [M_total][N], A [M_total][K], sa transposed with sa_stride >= M_total,
+ *   B [G][N][K], sb [G][ceil(N/128)][K/128], m_indices [M_total].
+ */
+DG_API dg_status dg_grouped_contiguous_nt(uint16_t* D, const uint8_t* A, const float* sa, int sa_stride,
+                                   const uint8_t* B, const float* sb, const int32_t* m_indices,
+                                   int M_total, int N, int K, int G, void* stream);
+
+/*
+ * Grouped GEMM, masked layout (section "分组 GEMM（掩码布局）"): for decoding
+ * under CUDA graphs, where the host does not know how many rows each group
+ * holds.  masked_m[g] (int32, device) rows of group g are computed; rows
+ * masked_m[g] .. M_max-1 of D[g] are left untouched.  The launch does not
+ * depend on masked_m.
+ *   D [G][M_max][N], A [G][M_max][K],
+ *   sa [G][K/128][sa_stride] (transposed per group, sa_stride >= M_max),
+ *   B [G][N][K], sb [G][ceil(N/128)][K/128], masked_m [G].
+ *   expected_m  host hint of the typical masked_m (<= 0: unknown); it may
+ *               change the tile shape chosen, never the result.
+ */
+DG_API dg_status dg_grouped_masked_nt(uint16_t* D, const uint8_t* A, const float* sa, int sa_stride,
+                               const uint8_t* B, const float* sb, const int32_t* masked_m,
+                               int G, int M_max, int N, int K, int expected_m, void* stream);
+
+/* Utility functions (section "工具函数" (utility functions) of the same page). */
+
+/* Cap the number of SMs the persistent kernels use (n <= 0: all SMs). */
+DG_API void dg_set_num_sms(int n);
+/* Current cap; the device's SM count when no cap is set (0 without a GPU). */
+DG_API int dg_get_num_sms(void);
+/* Row alignment every group segment needs in the contiguous layout (128). */
+DG_API int dg_get_m_alignment_for_contiguous_layout(void);
+/* x rounded up so that x*elem_bytes is a multiple of 16 bytes (TMA stride rule). */
+DG_API int dg_get_tma_aligned_size(int x, int elem_bytes);
+
+/* Reads the device error word of the current device, clears it, and stores it
+ * in *code.  Synchronises the device first; meant for tests and debugging. */
+DG_API dg_status dg_get_device_error(int* code);
+
+/* Static text for a status code. */
+DG_API const char* dg_status_string(dg_status s);
+/* Text describing the last failing call on this host thread ("" if none). */
+DG_API const char* dg_last_error_message(void);
+
+/*
+ * Launch plan (host only, no GPU needed): what a call with these sizes would
+ * launch.  mode: 0 dense, 1 contiguous, 2 masked.  rows = M (dense), M_total
+ * (contiguous) or M_max (masked).  Returns DG_ERR_INVALID_ARG for bad sizes.
+ */
+typedef struct dg_plan {
+    int block_m;      /* output rows per tile (tcgen05 M)                       */
+    int block_n;      /* output columns per tile (tcgen05 N)                     */
+    int stages;       /* depth of the shared-memory operand ring                 */
+    int m_blocks;     /* tiles along M (masked: worst case, G*ceil(M_max/BM))    */
+    int n_blocks;     /* tiles along N                                           */
+    int tiles;        /* m_blocks * n_blocks                                     */
+    int grid;         /* persistent CTAs launched                                */
+    int smem_bytes;   /* dynamic shared memory per CTA                           */
+} dg_plan;
+
+DG_API dg_status dg_make_plan(int mode, int rows, int N, int K, int G, int num_sms, dg_plan* out);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DG_H_ */

@@ -1,0 +1,171 @@
+"""Python binding of the B200 FP8 block-scaled NT GEMM library (libdg.so).
+
+Argument marshalling only: every function here forwards torch tensors' device
+pointers, their sizes and the current CUDA stream to the C ABI of
+``include/dg.h`` with the same name.  All arithmetic runs in the sm_100a kernels
+of ``libdg.so``; there is no fallback.  If the library is missing the first call
+raises ``RuntimeError`` (build it with ``__graft_entry__.build()`` or
+``python -m moe_grouped_gemm_weight_b200.build``).
+
+Layouts (see include/dg.h):
+  A   uint8 / float8_e4m3fn [M, K]          (masked: [G, M_max, K])
+  sa  float32, transposed: sa[kb*sa_stride + m] (masked: per group blocks)
+  B   uint8 / float8_e4m3fn [N, K] or [G, N, K]
+  sb  float32 [ceil(N/128), K/128] or [G, ceil(N/128), K/128]
+  D   bfloat16 [M, N]                        (masked: [G, M_max, N])
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libdg.so")
+
+DG_OK, DG_ERR_INVALID_ARG, DG_ERR_UNSUPPORTED, DG_ERR_MISALIGNED, DG_ERR_CUDA = range(5)
+DG_DEVERR_TIMEOUT, DG_DEVERR_BAD_M_INDEX, DG_DEVERR_BAD_MASKED_M = 1, 2, 4
+
+_lock = threading.Lock()
+_lib = None
+
+
+class DGError(RuntimeError):
+    def __init__(self, func: str, status: int, message: str):
+        super().__init__(f"{func}: {message} (status {status})")
+        self.status = status
+
+
+class Plan(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int) for n in
+                ("block_m", "block_n", "stages", "m_blocks", "n_blocks", "tiles", "grid", "smem_bytes")]
+
+    def as_dict(self) -> dict:
+        return {n: getattr(self, n) for n, _ in self._fields_}
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libdg.so (raises RuntimeError if it has not been built)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise RuntimeError(f"CUDA library {LIB_PATH} is missing: run __graft_entry__.build() first")
+            L = ctypes.CDLL(LIB_PATH)
+            P, I = ctypes.c_void_p, ctypes.c_int
+            L.dg_fp8_gemm_nt.restype = I
+            L.dg_fp8_gemm_nt.argtypes = [P, P, P, I, P, P, I, I, I, P]
+            L.dg_grouped_contiguous_nt.restype = I
+            L.dg_grouped_contiguous_nt.argtypes = [P, P, P, I, P, P, P, I, I, I, I, P]
+            L.dg_grouped_masked_nt.restype = I
+            L.dg_grouped_masked_nt.argtypes = [P, P, P, I, P, P, P, I, I, I, I, I, P]
+            L.dg_set_num_sms.restype = None
+            L.dg_set_num_sms.argtypes = [I]
+            L.dg_get_num_sms.restype = I
+            L.dg_get_num_sms.argtypes = []
+            L.dg_get_m_alignment_for_contiguous_layout.restype = I
+            L.dg_get_m_alignment_for_contiguous_layout.argtypes = []
+            L.dg_get_tma_aligned_size.restype = I
+            L.dg_get_tma_aligned_size.argtypes = [I, I]
+            L.dg_get_device_error.restype = I
+            L.dg_get_device_error.argtypes = [ctypes.POINTER(I)]
+            L.dg_status_string.restype = ctypes.c_char_p
+            L.dg_status_string.argtypes = [I]
+            L.dg_last_error_message.restype = ctypes.c_char_p
+            L.dg_last_error_message.argtypes = []
+            L.dg_make_plan.restype = I
+            L.dg_make_plan.argtypes = [I, I, I, I, I, I, ctypes.POINTER(Plan)]
+            _lib = L
+    return _lib
+
+
+def _check(func: str, status: int) -> None:
+    if status != DG_OK:
+        L = lib()
+        msg = L.dg_last_error_message().decode() or L.dg_status_string(status).decode()
+        raise DGError(func, status, msg)
+
+
+def _ptr(t) -> int:
+    return 0 if t is None else int(t.data_ptr())
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        import torch
+        return int(torch.cuda.current_stream().cuda_stream)
+    return int(stream if isinstance(stream, int) else stream.cuda_stream)
+
+
+def dg_fp8_gemm_nt(D, A, sa, sa_stride: int, B, sb, stream=None) -> None:
+    """Dense D[M,N] = scaled A[M,K] . B[N,K]^T (sizes taken from A and B)."""
+    M, K = A.shape[-2], A.shape[-1]
+    N = B.shape[-2]
+    _check("dg_fp8_gemm_nt", lib().dg_fp8_gemm_nt(_ptr(D), _ptr(A), _ptr(sa), int(sa_stride), _ptr(B), _ptr(sb),
+                                                  M, N, K, _stream(stream)))
+
+
+def dg_grouped_contiguous_nt(D, A, sa, sa_stride: int, B, sb, m_indices, stream=None) -> None:
+    """Contiguous-layout grouped GEMM; B is [G,N,K], m_indices int32 [M_total]."""
+    M, K = A.shape[-2], A.shape[-1]
+    G, N = B.shape[0], B.shape[1]
+    _check("dg_grouped_contiguous_nt",
+           lib().dg_grouped_contiguous_nt(_ptr(D), _ptr(A), _ptr(sa), int(sa_stride), _ptr(B), _ptr(sb),
+                                          _ptr(m_indices), M, N, K, G, _stream(stream)))
+
+
+def dg_grouped_masked_nt(D, A, sa, sa_stride: int, B, sb, masked_m, expected_m: int = 0, stream=None) -> None:
+    """Masked-layout grouped GEMM; A is [G,M_max,K], masked_m int32 [G] on the device."""
+    G, Mmax, K = A.shape
+    N = B.shape[1]
+    _check("dg_grouped_masked_nt",
+           lib().dg_grouped_masked_nt(_ptr(D), _ptr(A), _ptr(sa), int(sa_stride), _ptr(B), _ptr(sb),
+                                      _ptr(masked_m), G, Mmax, N, K, int(expected_m), _stream(stream)))
+
+
+def dg_set_num_sms(n: int) -> None:
+    lib().dg_set_num_sms(int(n))
+
+
+def dg_get_num_sms() -> int:
+    return int(lib().dg_get_num_sms())
+
+
+def dg_get_m_alignment_for_contiguous_layout() -> int:
+    return int(lib().dg_get_m_alignment_for_contiguous_layout())
+
+
+def dg_get_tma_aligned_size(x: int, elem_bytes: int) -> int:
+    return int(lib().dg_get_tma_aligned_size(int(x), int(elem_bytes)))
+
+
+def dg_get_device_error() -> int:
+    code = ctypes.c_int(0)
+    _check("dg_get_device_error", lib().dg_get_device_error(ctypes.byref(code)))
+    return int(code.value)
+
+
+def dg_make_plan(mode: int, rows: int, N: int, K: int, G: int, num_sms: int) -> dict:
+    pl = Plan()
+    _check("dg_make_plan", lib().dg_make_plan(int(mode), int(rows), int(N), int(K), int(G), int(num_sms),
+                                              ctypes.byref(pl)))
+    return pl.as_dict()
+
+
+def dg_status_string(status: int) -> str:
+    return lib().dg_status_string(int(status)).decode()
+
+
+def dg_get_col_major_tma_aligned_tensor(s):
+    """[M, nkb] (or [G, M, nkb]) float32 scales -> (flat transposed TMA-aligned tensor, sa_stride).
+
+    Layout helper for callers (the pages' get_col_major_tma_aligned_tensor);
+    runs as torch tensor ops outside the timed path."""
+    import torch
+    grouped = s.dim() == 3
+    s3 = s if grouped else s.unsqueeze(0)
+    G, M, nkb = s3.shape
+    stride = dg_get_tma_aligned_size(M, 4)
+    out = torch.zeros(G, nkb, stride, dtype=torch.float32, device=s.device)
+    out[:, :, :M] = s3.transpose(1, 2)
+    return out.reshape(-1).contiguous(), stride

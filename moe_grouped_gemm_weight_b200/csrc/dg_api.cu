@@ -1,0 +1,357 @@
+// dg_api.cu -- host side of the C ABI declared in include/dg.h: argument
+// validation, the launch plan (tile shape, ring depth, grid), TMA tensor-map
+// encoding and kernel dispatch.  Nothing here allocates device memory, reads
+// device memory or synchronises, except dg_get_device_error().
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "dg.h"
+#include "dg_kernel.cuh"
+
+namespace {
+
+thread_local char g_msg[512] = "";
+std::atomic<int> g_num_sms_cap{0};
+
+dg_status fail(dg_status s, const char* fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_msg, sizeof(g_msg), fmt, ap);
+    va_end(ap);
+    return s;
+}
+
+dg_status ok() {
+    g_msg[0] = '\0';
+    return DG_OK;
+}
+
+int cdiv(int a, int b) { return (a + b - 1) / b; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// ------------------------------------------------------------- devices ----
+
+constexpr int kMaxDevices = 64;
+std::atomic<int> g_sm_count[kMaxDevices];
+
+int device_sm_count(int* dev_out = nullptr) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        return 0;
+    }
+    if (dev_out) *dev_out = dev;
+    if (dev < 0 || dev >= kMaxDevices) return 0;
+    int n = g_sm_count[dev].load();
+    if (n == 0) {
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+            cudaGetLastError();
+            return 0;
+        }
+        g_sm_count[dev].store(n);
+    }
+    return n;
+}
+
+// ------------------------------------------------------ tensor maps ----
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+        else
+            cudaGetLastError();
+    });
+    return fn;
+}
+
+// K-major e4m3 operand: dims (K, rows[, groups]), box (128, box_rows[, 1]),
+// 128-byte swizzle, zero fill outside the tensor.
+dg_status make_operand_map(CUtensorMap* tm, const void* base, int K, int rows, int groups, int box_rows,
+                           bool three_d) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return fail(DG_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+    cuuint64_t dims[3] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows),
+                          static_cast<cuuint64_t>(groups)};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(K) * rows};
+    cuuint32_t box[3] = {static_cast<cuuint32_t>(dg::kBK), static_cast<cuuint32_t>(box_rows), 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, three_d ? 3 : 2, const_cast<void*>(base), dims, strides, box,
+                    estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(DG_ERR_CUDA, "cuTensorMapEncodeTiled failed (CUresult %d)", static_cast<int>(r));
+    return DG_OK;
+}
+
+// ------------------------------------------------------------ planning ----
+
+struct Choice {
+    int bn;
+    int stages;
+};
+
+// Ring depth: as many stages as fit in 227 KiB of shared memory, at most 8.
+template <int BN>
+constexpr int max_stages() {
+    int s = 8;
+    while (s > 2 && dg::smem_bytes<BN, 8>() - (8 - s) * (dg::kTileABytes + BN * dg::kBK) > 227 * 1024) --s;
+    return s;
+}
+
+int waves_cost(int tiles, int sms) { return cdiv(tiles, sms); }
+
+// Tile width: the widest N tile (fewer A re-reads, more tensor work per byte
+// of shared memory) unless a narrower one spreads the problem over more SMs
+// -- the point of the "non-aligned block size" optimisation on the DeepGEMM
+// README page (section "非对齐的块大小"), here restricted to N tiles that the
+// promotion warps split into 32-column TMEM loads.
+Choice choose(int m_blocks, int N, int num_sms) {
+    const int cands[2] = {128, 64};
+    Choice best{128, max_stages<128>()};
+    long best_cost = -1;
+    for (int bn : cands) {
+        const int tiles = m_blocks * cdiv(N, bn);
+        // Cost model: waves of tiles times the per-tile time, taken as
+        // proportional to the tile width (both operands stream per K block).
+        const long cost = static_cast<long>(waves_cost(tiles, num_sms)) * (bn + 128);
+        if (best_cost < 0 || cost < best_cost) {
+            best_cost = cost;
+            best.bn = bn;
+        }
+    }
+    best.stages = best.bn == 128 ? max_stages<128>() : max_stages<64>();
+    return best;
+}
+
+int plan_smem(const Choice& c) {
+    return c.bn == 128 ? dg::smem_bytes<128, 8>() - (8 - c.stages) * (dg::kTileABytes + 128 * dg::kBK)
+                       : dg::smem_bytes<64, 8>() - (8 - c.stages) * (dg::kTileABytes + 64 * dg::kBK);
+}
+
+dg_status check_sizes(int mode, int rows, int N, int K, int G) {
+    if (rows < 0 || N <= 0 || K <= 0 || G <= 0)
+        return fail(DG_ERR_INVALID_ARG, "sizes must be positive (rows=%d N=%d K=%d G=%d)", rows, N, K, G);
+    if (K % 128 != 0) return fail(DG_ERR_UNSUPPORTED, "K=%d is not a multiple of 128", K);
+    if (N % 8 != 0) return fail(DG_ERR_UNSUPPORTED, "N=%d is not a multiple of 8", N);
+    if (mode == 1 && rows % dg::kBM != 0)
+        return fail(DG_ERR_INVALID_ARG, "contiguous layout: M_total=%d is not a multiple of %d", rows, dg::kBM);
+    if (mode == 2 && G > dg::kMaxMaskedGroups)
+        return fail(DG_ERR_UNSUPPORTED, "masked layout supports at most %d groups (G=%d)", dg::kMaxMaskedGroups, G);
+    const long long a_elems = static_cast<long long>(rows) * K * (mode == 2 ? G : 1);
+    const long long b_elems = static_cast<long long>(G) * N * K;
+    if (a_elems >= (1ll << 40) || b_elems >= (1ll << 40) || static_cast<long long>(rows) * G >= (1ll << 31))
+        return fail(DG_ERR_UNSUPPORTED, "problem too large");
+    return DG_OK;
+}
+
+dg_status plan(int mode, int rows, int N, int K, int G, int num_sms, dg_plan* out) {
+    dg_status s = check_sizes(mode, rows, N, K, G);
+    if (s != DG_OK) return s;
+    if (num_sms <= 0) return fail(DG_ERR_INVALID_ARG, "num_sms must be positive");
+    const int m_blocks = (mode == 2) ? G * cdiv(rows, dg::kBM) : cdiv(rows, dg::kBM);
+    // Masked: the host does not know masked_m, so plan for every group being
+    // half full (or for expected_m, see dg_grouped_masked_nt).
+    const Choice c = choose(m_blocks, N, num_sms);
+    out->block_m = dg::kBM;
+    out->block_n = c.bn;
+    out->stages = c.stages;
+    out->m_blocks = m_blocks;
+    out->n_blocks = cdiv(N, c.bn);
+    out->tiles = m_blocks * out->n_blocks;
+    out->grid = (mode == 2) ? num_sms : (out->tiles < num_sms ? out->tiles : num_sms);
+    out->smem_bytes = plan_smem(c);
+    return DG_OK;
+}
+
+// ------------------------------------------------------------ launch ----
+
+template <int BN, int STAGES, int MODE>
+dg_status launch_one(const dg::Params& p, const CUtensorMap& ta, const CUtensorMap& tb, int grid,
+                     cudaStream_t stream) {
+    constexpr int smem = dg::smem_bytes<BN, STAGES>();
+    static_assert(smem <= 227 * 1024, "shared memory budget exceeded");
+    auto kern = dg::fp8_gemm_kernel<BN, STAGES, MODE>;
+    static std::atomic<int> attr_set[kMaxDevices];
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev >= 0 && dev < kMaxDevices && !attr_set[dev].load()) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+            return fail(DG_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(cudaGetLastError()));
+        attr_set[dev].store(1);
+    }
+    kern<<<grid, dg::kThreads, smem, stream>>>(p, ta, tb);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(DG_ERR_CUDA, "kernel launch failed: %s", cudaGetErrorString(e));
+    return ok();
+}
+
+template <int MODE>
+dg_status dispatch(const dg_plan& pl, const dg::Params& p, const CUtensorMap& ta, const CUtensorMap& tb,
+                   cudaStream_t stream) {
+    if (pl.block_n == 128) {
+        constexpr int S = max_stages<128>();
+        return launch_one<128, S, MODE>(p, ta, tb, pl.grid, stream);
+    }
+    constexpr int S = max_stages<64>();
+    return launch_one<64, S, MODE>(p, ta, tb, pl.grid, stream);
+}
+
+int effective_sms() {
+    const int dev_sms = device_sm_count();
+    const int cap = g_num_sms_cap.load();
+    if (cap > 0 && (dev_sms == 0 || cap < dev_sms)) return cap;
+    return dev_sms;
+}
+
+dg_status common_checks(const void* D, const void* A, const float* sa, int sa_stride, const void* B, const float* sb,
+                        int rows) {
+    if (!D || !A || !sa || !B || !sb) return fail(DG_ERR_INVALID_ARG, "null tensor pointer");
+    if (!aligned16(D) || !aligned16(A) || !aligned16(sa) || !aligned16(B) || !aligned16(sb))
+        return fail(DG_ERR_MISALIGNED, "tensor pointers must be 16-byte aligned");
+    if (sa_stride < rows || sa_stride % 4 != 0)
+        return fail(DG_ERR_INVALID_ARG, "sa_stride=%d must be >= %d and a multiple of 4", sa_stride, rows);
+    return DG_OK;
+}
+
+dg::Params make_params(uint16_t* D, const float* sa, int sa_stride, const float* sb, int rows, int N, int K, int G,
+                       const dg_plan& pl) {
+    dg::Params p{};
+    p.D = D;
+    p.sa = sa;
+    p.sb = sb;
+    p.sa_stride = sa_stride;
+    p.M = rows;
+    p.N = N;
+    p.K = K;
+    p.G = G;
+    p.nkb = K / dg::kBK;
+    p.nbn = cdiv(N, 128);
+    p.n_blocks = pl.n_blocks;
+    p.m_blocks = pl.m_blocks;
+    p.raster = 8;
+    return p;
+}
+
+}  // namespace
+
+extern "C" {
+
+dg_status dg_fp8_gemm_nt(uint16_t* D, const uint8_t* A, const float* sa, int sa_stride, const uint8_t* B,
+                         const float* sb, int M, int N, int K, void* stream) {
+    dg_status s = check_sizes(0, M, N, K, 1);
+    if (s != DG_OK) return s;
+    if ((s = common_checks(D, A, sa, sa_stride, B, sb, M)) != DG_OK) return s;
+    if (M == 0) return ok();
+    const int sms = effective_sms();
+    if (sms <= 0) return fail(DG_ERR_CUDA, "no CUDA device");
+    dg_plan pl;
+    if ((s = plan(0, M, N, K, 1, sms, &pl)) != DG_OK) return s;
+    CUtensorMap ta, tb;
+    if ((s = make_operand_map(&ta, A, K, M, 1, dg::kBM, false)) != DG_OK) return s;
+    if ((s = make_operand_map(&tb, B, K, N, 1, pl.block_n, true)) != DG_OK) return s;
+    dg::Params p = make_params(D, sa, sa_stride, sb, M, N, K, 1, pl);
+    return dispatch<dg::kDense>(pl, p, ta, tb, static_cast<cudaStream_t>(stream));
+}
+
+dg_status dg_grouped_contiguous_nt(uint16_t* D, const uint8_t* A, const float* sa, int sa_stride, const uint8_t* B,
+                                   const float* sb, const int32_t* m_indices, int M_total, int N, int K, int G,
+                                   void* stream) {
+    dg_status s = check_sizes(1, M_total, N, K, G);
+    if (s != DG_OK) return s;
+    if ((s = common_checks(D, A, sa, sa_stride, B, sb, M_total)) != DG_OK) return s;
+    if (!m_indices) return fail(DG_ERR_INVALID_ARG, "null m_indices");
+    if (M_total == 0) return ok();
+    const int sms = effective_sms();
+    if (sms <= 0) return fail(DG_ERR_CUDA, "no CUDA device");
+    dg_plan pl;
+    if ((s = plan(1, M_total, N, K, G, sms, &pl)) != DG_OK) return s;
+    CUtensorMap ta, tb;
+    if ((s = make_operand_map(&ta, A, K, M_total, 1, dg::kBM, false)) != DG_OK) return s;
+    if ((s = make_operand_map(&tb, B, K, N, G, pl.block_n, true)) != DG_OK) return s;
+    dg::Params p = make_params(D, sa, sa_stride, sb, M_total, N, K, G, pl);
+    p.m_indices = m_indices;
+    return dispatch<dg::kContiguous>(pl, p, ta, tb, static_cast<cudaStream_t>(stream));
+}
+
+dg_status dg_grouped_masked_nt(uint16_t* D, const uint8_t* A, const float* sa, int sa_stride, const uint8_t* B,
+                               const float* sb, const int32_t* masked_m, int G, int M_max, int N, int K,
+                               int expected_m, void* stream) {
+    (void)expected_m;
+    dg_status s = check_sizes(2, M_max, N, K, G);
+    if (s != DG_OK) return s;
+    if ((s = common_checks(D, A, sa, sa_stride, B, sb, M_max)) != DG_OK) return s;
+    if (!masked_m) return fail(DG_ERR_INVALID_ARG, "null masked_m");
+    if (M_max == 0) return ok();
+    const int sms = effective_sms();
+    if (sms <= 0) return fail(DG_ERR_CUDA, "no CUDA device");
+    dg_plan pl;
+    if ((s = plan(2, M_max, N, K, G, sms, &pl)) != DG_OK) return s;
+    CUtensorMap ta, tb;
+    if ((s = make_operand_map(&ta, A, K, M_max, G, dg::kBM, true)) != DG_OK) return s;
+    if ((s = make_operand_map(&tb, B, K, N, G, pl.block_n, true)) != DG_OK) return s;
+    dg::Params p = make_params(D, sa, sa_stride, sb, M_max, N, K, G, pl);
+    p.masked_m = masked_m;
+    return dispatch<dg::kMasked>(pl, p, ta, tb, static_cast<cudaStream_t>(stream));
+}
+
+void dg_set_num_sms(int n) { g_num_sms_cap.store(n > 0 ? n : 0); }
+
+int dg_get_num_sms(void) { return effective_sms(); }
+
+int dg_get_m_alignment_for_contiguous_layout(void) { return dg::kBM; }
+
+int dg_get_tma_aligned_size(int x, int elem_bytes) {
+    if (x < 0 || elem_bytes <= 0 || 16 % elem_bytes != 0) return -1;
+    const int per = 16 / elem_bytes;
+    return cdiv(x, per) * per;
+}
+
+dg_status dg_get_device_error(int* code) {
+    if (!code) return fail(DG_ERR_INVALID_ARG, "null code pointer");
+    cudaError_t e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) return fail(DG_ERR_CUDA, "cudaDeviceSynchronize: %s", cudaGetErrorString(e));
+    unsigned int v = 0, zero = 0;
+    e = cudaMemcpyFromSymbol(&v, dg::g_dg_error, sizeof(v));
+    if (e == cudaSuccess) e = cudaMemcpyToSymbol(dg::g_dg_error, &zero, sizeof(zero));
+    if (e != cudaSuccess) return fail(DG_ERR_CUDA, "reading the device error word: %s", cudaGetErrorString(e));
+    *code = static_cast<int>(v);
+    return ok();
+}
+
+const char* dg_status_string(dg_status s) {
+    switch (s) {
+        case DG_OK: return "ok";
+        case DG_ERR_INVALID_ARG: return "invalid argument";
+        case DG_ERR_UNSUPPORTED: return "unsupported shape or layout";
+        case DG_ERR_MISALIGNED: return "misaligned pointer";
+        case DG_ERR_CUDA: return "CUDA error";
+    }
+    return "unknown status";
+}
+
+const char* dg_last_error_message(void) { return g_msg; }
+
+dg_status dg_make_plan(int mode, int rows, int N, int K, int G, int num_sms, dg_plan* out) {
+    if (!out) return fail(DG_ERR_INVALID_ARG, "null plan pointer");
+    if (mode < 0 || mode > 2) return fail(DG_ERR_INVALID_ARG, "mode must be 0, 1 or 2");
+    if (mode == 0 && G != 1) return fail(DG_ERR_INVALID_ARG, "dense mode needs G == 1");
+    return plan(mode, rows, N, K, G, num_sms, out);
+}
+
+}  // extern "C"

@@ -1,0 +1,137 @@
+"""Host-side tests of the C ABI (no GPU needed): the library loads, exports every
+symbol include/dg.h declares, its utilities and launch plan follow the pages'
+rules, and bad arguments are rejected synchronously before any CUDA call."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import moe_grouped_gemm_weight_b200 as dg
+from moe_grouped_gemm_weight_b200 import build as dgbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "dg.h")
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built_library():
+    dgbuild.build()
+    yield
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"^DG_API\s+[\w\s\*]+?\b(dg_\w+)\s*\(", text, re.M)))
+
+
+def test_header_declares_the_three_gemms_and_utilities():
+    names = declared_functions()
+    for n in ["dg_fp8_gemm_nt", "dg_grouped_contiguous_nt", "dg_grouped_masked_nt", "dg_set_num_sms",
+              "dg_get_num_sms", "dg_get_m_alignment_for_contiguous_layout", "dg_get_tma_aligned_size",
+              "dg_get_device_error", "dg_status_string", "dg_last_error_message", "dg_make_plan"]:
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol():
+    L = ctypes.CDLL(dg.LIB_PATH)
+    missing = [n for n in declared_functions() if not hasattr(L, n)]
+    assert not missing, missing
+
+
+def test_library_exports_nothing_undeclared():
+    out = os.popen(f"nm -D --defined-only {dg.LIB_PATH}").read()
+    exported = {l.split()[-1] for l in out.splitlines() if " T " in l and l.split()[-1].startswith("dg")}
+    assert exported == set(declared_functions())
+
+
+def test_library_does_not_link_the_oracle():
+    out = os.popen(f"ldd {dg.LIB_PATH}").read() + os.popen(f"nm -D {dg.LIB_PATH}").read()
+    assert "oracle" not in out and "dgo_" not in out
+
+
+def test_utilities():
+    assert dg.dg_get_m_alignment_for_contiguous_layout() == 128
+    assert dg.dg_get_tma_aligned_size(64, 4) == 64
+    assert dg.dg_get_tma_aligned_size(65, 4) == 68
+    assert dg.dg_get_tma_aligned_size(1, 4) == 4
+    assert dg.dg_get_tma_aligned_size(3, 2) == 8
+    assert dg.dg_get_tma_aligned_size(17, 1) == 32
+    assert dg.dg_get_tma_aligned_size(0, 4) == 0
+    assert dg.dg_status_string(0) == "ok"
+    assert "invalid" in dg.dg_status_string(1)
+
+
+def test_plan_reproduces_the_pages_block_count_arithmetic():
+    # README page, section "非对齐的块大小": M=256, N=7168 with 128x128 blocks
+    # gives (256/128)*(7168/128) = 112 tiles, which leaves SMs of a 132-SM part
+    # idle.  The plan keeps the tile arithmetic exact.
+    p = dg.dg_make_plan(0, 256, 7168, 7168, 1, 132)
+    assert p["block_m"] == 128
+    assert p["m_blocks"] == 2
+    assert p["tiles"] == p["m_blocks"] * p["n_blocks"]
+    assert p["n_blocks"] == -(-7168 // p["block_n"])
+    if p["block_n"] == 128:
+        assert p["tiles"] == 112
+
+
+@pytest.mark.parametrize("mode,rows,N,K,G", [(0, 64, 2112, 7168, 1), (0, 4096, 7168, 16384, 1),
+                                            (1, 32768, 4096, 7168, 4), (2, 256, 4096, 7168, 4)])
+def test_plan_is_consistent(mode, rows, N, K, G):
+    p = dg.dg_make_plan(mode, rows, N, K, G, 148)
+    assert p["block_n"] in (64, 128, 192, 256)
+    assert p["n_blocks"] == -(-N // p["block_n"])
+    mb = -(-rows // 128) * (G if mode == 2 else 1)
+    assert p["m_blocks"] == mb
+    assert p["tiles"] == mb * p["n_blocks"]
+    assert 1 <= p["grid"] <= 148
+    assert p["smem_bytes"] <= 227 * 1024
+    assert p["stages"] >= 2
+
+
+@pytest.mark.parametrize("args,expect", [
+    ((0, 64, 2112, 7100, 1), dg.DG_ERR_UNSUPPORTED),  # K % 128
+    ((0, 64, 2110, 7168, 1), dg.DG_ERR_UNSUPPORTED),  # N % 8
+    ((0, -1, 64, 128, 1), dg.DG_ERR_INVALID_ARG),
+    ((1, 130, 64, 128, 2), dg.DG_ERR_INVALID_ARG),    # contiguous M_total % 128
+    ((2, 64, 64, 128, 5000), dg.DG_ERR_UNSUPPORTED),  # too many masked groups
+    ((3, 64, 64, 128, 1), dg.DG_ERR_INVALID_ARG),     # bad mode
+])
+def test_plan_rejects_bad_sizes(args, expect):
+    with pytest.raises(dg.DGError) as ei:
+        dg.dg_make_plan(*args, 148)
+    assert ei.value.status == expect
+
+
+def test_gemm_calls_reject_bad_arguments_without_touching_the_gpu():
+    L = dg.lib()
+    fake = 1 << 20  # never dereferenced: every call below fails validation first
+    st = L.dg_fp8_gemm_nt(fake, fake, fake, 64, fake, fake, 64, 64, 100, 0)
+    assert st == dg.DG_ERR_UNSUPPORTED and b"K=100" in L.dg_last_error_message()
+    assert L.dg_fp8_gemm_nt(0, fake, fake, 64, fake, fake, 64, 64, 128, 0) == dg.DG_ERR_INVALID_ARG
+    assert L.dg_fp8_gemm_nt(fake + 4, fake, fake, 64, fake, fake, 64, 64, 128, 0) == dg.DG_ERR_MISALIGNED
+    assert L.dg_fp8_gemm_nt(fake, fake, fake, 62, fake, fake, 64, 64, 128, 0) == dg.DG_ERR_INVALID_ARG
+    assert L.dg_fp8_gemm_nt(fake, fake, fake, 66, fake, fake, 64, 64, 128, 0) == dg.DG_ERR_INVALID_ARG
+    assert L.dg_grouped_contiguous_nt(fake, fake, fake, 128, fake, fake, 0, 128, 64, 128, 2, 0) == \
+        dg.DG_ERR_INVALID_ARG
+    assert L.dg_grouped_contiguous_nt(fake, fake, fake, 200, fake, fake, fake, 200, 64, 128, 2, 0) == \
+        dg.DG_ERR_INVALID_ARG
+    assert L.dg_grouped_masked_nt(fake, fake, fake, 64, fake, fake, 0, 2, 64, 64, 128, 0, 0) == \
+        dg.DG_ERR_INVALID_ARG
+    assert L.dg_grouped_masked_nt(fake, fake, fake, 64, fake, fake, fake, 2, 64, 64, 128, 0, 0) != dg.DG_OK or \
+        dg.dg_get_num_sms() > 0
+
+
+def test_empty_problem_is_a_no_op():
+    L = dg.lib()
+    fake = 1 << 20
+    assert L.dg_fp8_gemm_nt(fake, fake, fake, 0, fake, fake, 0, 64, 128, 0) == dg.DG_OK
+
+
+def test_binding_fails_loudly_when_library_missing(tmp_path, monkeypatch):
+    import importlib
+    mod = importlib.import_module("moe_grouped_gemm_weight_b200")
+    monkeypatch.setattr(mod, "_lib", None)
+    monkeypatch.setattr(mod, "LIB_PATH", str(tmp_path / "missing.so"))
+    with pytest.raises(RuntimeError, match="missing"):
+        mod.dg_get_num_sms()
