@@ -1,0 +1,454 @@
+"""Benchmark of the B200 FP8 block-scaled NT GEMM (dense sweep + grouped forms).
+
+Usage:  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One STEP is one pass over the dense sweep of the DeepGEMM performance table:
+M in {64, 128, 4096} x (N, K) in {(2112,7168), (24576,1536), (32768,512),
+(7168,16384), (4096,7168), (7168,2048)}, e4m3 inputs with 1x128 / 128x128 FP32
+scales, bf16 output -- 18 GEMMs through the C ABI.  Before every GEMM a 512 MiB
+buffer is overwritten (L2 flush, untimed); each GEMM is timed with CUDA events
+on the stream it is launched on.  ``value`` is the aggregate TFLOP/s of the
+sweep (sum of flops / sum of kernel times), max over ranks for N > 1 (each
+rank runs the same sweep on its own GPU: weak scaling, no collective on the
+data path).  The grouped contiguous and masked workloads are timed the same way
+and reported under ``grouped``.  ``e2e`` is the same sweep measured around
+pinned-host -> device copies of every input, the GEMM and the device -> host
+copy of D.  ``cpu_baseline`` times the CPU oracle on a bounded row sample.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+import workloads as wl  # noqa: E402
+
+SPEC_FP8_TFLOPS = 4500.0    # B200 dense FP8 datasheet figure
+SPEC_HBM_GBS = 8000.0       # HBM3e datasheet figure used by the target
+FP8_PER_BF16 = 2.0          # nominal dense FP8 : BF16 tensor ratio (4.5 : 2.25 PF)
+L2_FLUSH_BYTES = 512 << 20
+
+
+def load_peaks() -> dict:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            m = json.load(f)
+        return {"hbm_gbs": float(m["hbm_gbs"]), "bf16_tflops": float(m["bf16_tflops"]),
+                "bf16_tflops_sustained": float(m.get("bf16_tflops_sustained", m["bf16_tflops"])),
+                "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+# ------------------------------------------------------------ distributed ---
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", str(rank)))
+    return rank, world, local
+
+
+def dist_init(world: int, backend: str):
+    if world > 1 and not torch.distributed.is_initialized():
+        import datetime
+        torch.distributed.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+
+
+def barrier(world: int):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate(total_flops_per_rank: float, seconds_max: float, world: int) -> float:
+    """Whole-job TFLOP/s: the work of all ranks over the slowest rank's time."""
+    return total_flops_per_rank * world / seconds_max / 1e12
+
+
+# ---------------------------------------------------------------- clocks ----
+
+class ClockSampler:
+    """Samples SM clock, max clock, power and clock-event reasons every 20 ms
+    through NVML (read-only queries, the data nvidia-smi prints) while active."""
+
+    REASONS = {"sw_power_cap": "nvmlClocksEventReasonSwPowerCap",
+               "hw_slowdown": "nvmlClocksEventReasonHwSlowdown",
+               "hw_thermal_slowdown": "nvmlClocksEventReasonHwThermalSlowdown",
+               "sw_thermal_slowdown": "nvmlClocksEventReasonSwThermalSlowdown",
+               "hw_power_brake_slowdown": "nvmlClocksEventReasonHwPowerBrakeSlowdown"}
+
+    def __init__(self, gpu_index: int, period_s: float = 0.02):
+        self.gpu, self.period = gpu_index, period_s
+        self.samples, self.thread, self.stop = [], None, None
+        self.nvml = None
+
+    def __enter__(self):
+        import threading
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+            idx = int(vis.split(",")[self.gpu]) if vis and vis.split(",")[0].isdigit() else self.gpu
+            self.handle = pynvml.nvmlDeviceGetHandleByIndex(idx)
+            self.nvml = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.handle, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self.nvml = None
+            return self
+        self.stop = threading.Event()
+
+        def loop():
+            n = self.nvml
+            while not self.stop.is_set():
+                try:
+                    sm = n.nvmlDeviceGetClockInfo(self.handle, n.NVML_CLOCK_SM)
+                    rs = n.nvmlDeviceGetCurrentClocksEventReasons(self.handle)
+                    pw = n.nvmlDeviceGetPowerUsage(self.handle) / 1000.0
+                    self.samples.append((sm, rs, pw))
+                except Exception:
+                    pass
+                self.stop.wait(self.period)
+
+        self.thread = threading.Thread(target=loop, daemon=True)
+        self.thread.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.thread is not None:
+            self.stop.set()
+            self.thread.join(timeout=2)
+
+    def summary(self) -> dict:
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        n = self.nvml
+        reasons = sorted({name for _, rs, _ in self.samples for name, attr in self.REASONS.items()
+                          if rs & getattr(n, attr, 0)})
+        sm = [x[0] for x in self.samples]
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": self.max_mhz, "sm_mhz_min": min(sm),
+                "power_w_max": round(max(x[2] for x in self.samples), 1), "reasons": reasons,
+                "samples": len(self.samples), "source": "nvml, every 20 ms during the timed steps"}
+
+
+# ------------------------------------------------------------------ ours ----
+
+class Problem:
+    def __init__(self, case: wl.Case, dg):
+        self.case = case
+        self.dg = dg
+        c = case
+        if c.mode == "masked":
+            self.D = torch.empty(c.G, c.M, c.N, dtype=torch.bfloat16, device="cuda")
+        else:
+            self.D = torch.empty(c.M, c.N, dtype=torch.bfloat16, device="cuda")
+        self.flops = c.flops()
+        self.bytes = c.bytes()
+        mode = {"dense": 0, "contiguous": 1, "masked": 2}[c.mode]
+        self.plan = dg.dg_make_plan(mode, c.M, c.N, c.K, c.G, dg.dg_get_num_sms())
+        self.kernel = f"fp8_gemm_kernel<BN={self.plan['block_n']},STAGES={self.plan['stages']},{c.mode}>"
+
+    def run(self, case=None, D=None):
+        c = case or self.case
+        D = self.D if D is None else D
+        if c.mode == "dense":
+            self.dg.dg_fp8_gemm_nt(D, c.A, c.sa, c.sa_stride, c.B, c.sb)
+        elif c.mode == "contiguous":
+            self.dg.dg_grouped_contiguous_nt(D, c.A, c.sa, c.sa_stride, c.B, c.sb, c.m_indices)
+        else:
+            self.dg.dg_grouped_masked_nt(D, c.A, c.sa, c.sa_stride, c.B, c.sb, c.masked_m)
+
+
+def roof_time_s(flops, byts, tflops, gbs):
+    return max(flops / (tflops * 1e12), byts / (gbs * 1e9))
+
+
+def time_problems(problems, flush, reps: int):
+    """Per-problem list of kernel times (s), L2 flushed before every launch."""
+    stream = torch.cuda.current_stream()
+    times = [[] for _ in problems]
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in problems]
+    for _ in range(reps):
+        for i, p in enumerate(problems):
+            flush.zero_()
+            evs[i][0].record(stream)
+            p.run()
+            evs[i][1].record(stream)
+        torch.cuda.synchronize()
+        for i in range(len(problems)):
+            times[i].append(evs[i][0].elapsed_time(evs[i][1]) * 1e-3)
+    return times
+
+
+def oracle_rows_sample(c: wl.Case, nrows: int, salt: int = 0):
+    """A deterministic spread of nrows distinct row indices of a case."""
+    import numpy as np
+    n = min(nrows, c.M)
+    return np.array(sorted({(salt + i * 9973) % c.M for i in range(n)}), dtype=np.int64)
+
+
+def cpu_baseline(problems, budget_s: float = 15.0) -> dict:
+    """The CPU oracle, as it stands, on a bounded row sample of every shape.
+
+    The oracle parallelises over output rows, so each call gets one row per
+    host thread; calls repeat per shape until that shape's share of the budget
+    is spent."""
+    import oracle
+    threads = oracle.num_threads()
+    flops, t_total = 0.0, 0.0
+    sample = []
+    per_shape_budget = budget_s / len(problems)
+    for p in problems:
+        c = p.case
+        A, sa, B, sb = c.A.cpu().numpy(), c.sa.cpu().numpy(), c.B.cpu().numpy(), c.sb.cpu().numpy()
+        spent, nrows, calls = 0.0, 0, 0
+        while spent < per_shape_budget:
+            rows = oracle_rows_sample(c, threads, salt=calls)
+            t0 = time.perf_counter()
+            oracle.gemm_nt(A, sa, c.sa_stride, B, sb, c.M, c.N, c.K, rows=rows, want_d64=False, want_mag=False)
+            spent += time.perf_counter() - t0
+            nrows += len(rows)
+            calls += 1
+        flops += 2.0 * nrows * c.N * c.K
+        t_total += spent
+        sample.append(f"{c.M}x{c.N}x{c.K}:{nrows}rows")
+    return {"value": flops / t_total / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+            "sample": "all N columns of a few rows of every dense-sweep shape (" + ", ".join(sample) + ")",
+            "seconds": round(t_total, 2)}
+
+
+def run_ours(args, rank, world, local):
+    torch.cuda.set_device(local)
+    dist_init(world, "nccl")
+    from moe_grouped_gemm_weight_b200 import build as dgbuild
+    dgbuild.build()
+    import moe_grouped_gemm_weight_b200 as dg
+
+    peaks = load_peaks()
+    p_fp8_burst = peaks["bf16_tflops"] * FP8_PER_BF16
+    dev = torch.device("cuda", local)
+
+    shapes = wl.DENSE_SWEEP
+    if args.shape:
+        shapes = [tuple(int(x) for x in args.shape.lower().split("x"))]
+    problems = [Problem(wl.dense_case(m, n, k, seed=0, device="cuda"), dg) for (m, n, k) in shapes]
+    grouped = [] if args.no_grouped else [
+        Problem(wl.contiguous_case(device="cuda", seed=0, **wl.CONTIGUOUS_MAIN), dg),
+        Problem(wl.masked_case(device="cuda", seed=0, **wl.MASKED_MAIN), dg),
+        Problem(wl.masked_case(device="cuda", seed=0, **wl.MASKED_SINGLE), dg)]
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    step_flops = float(sum(p.flops for p in problems))
+
+    # warm-up (also first-call set-up of every kernel instance)
+    time_problems(problems + grouped, flush, max(args.warmup, 1))
+
+    # ---- timed region: exactly K steps ----
+    barrier(world)
+    torch.cuda.synchronize()
+    t_wall0 = time.perf_counter()
+    with ClockSampler(local) as clk:
+        times = time_problems(problems, flush, args.steps)
+        torch.cuda.synchronize()
+    t_wall = time.perf_counter() - t_wall0
+    barrier(world)
+    clocks = clk.summary()
+
+    kernel_s = sum(sum(t) for t in times)           # K steps of kernel time
+    kernel_s_max = max_over_ranks(kernel_s, world, dev)
+    value = aggregate(step_flops * args.steps, kernel_s_max, world)
+    ms_per_step = kernel_s_max / args.steps * 1e3
+
+    per_shape = []
+    for p, t in zip(problems, times):
+        tm = statistics.median(t)
+        c = p.case
+        per_shape.append({
+            "M": c.M, "N": c.N, "K": c.K, "us": round(tm * 1e6, 2),
+            "tflops": round(p.flops / tm / 1e12, 1), "gbs": round(p.bytes / tm / 1e9, 1),
+            "frac_roof_spec": round(roof_time_s(p.flops, p.bytes, SPEC_FP8_TFLOPS, SPEC_HBM_GBS) / tm, 3),
+            "frac_roof_measured": round(roof_time_s(p.flops, p.bytes, p_fp8_burst, peaks["hbm_gbs"]) / tm, 3),
+            "bound": "tensor" if p.flops / p_fp8_burst / 1e12 > p.bytes / peaks["hbm_gbs"] / 1e9 else "hbm",
+            "block_n": p.plan["block_n"],
+        })
+
+    # dominant kernel instance: the one with the largest share of step time
+    by_kernel = {}
+    for p, t in zip(problems, times):
+        d = by_kernel.setdefault(p.kernel, {"flops": 0.0, "bytes": 0.0, "s": 0.0, "launches": 0})
+        d["flops"] += p.flops * len(t)
+        d["bytes"] += p.bytes * len(t)
+        d["s"] += sum(t)
+        d["launches"] += len(t)
+    dom_name, dom = max(by_kernel.items(), key=lambda kv: kv[1]["s"])
+    tensor_bound = dom["flops"] / (p_fp8_burst * 1e12) > dom["bytes"] / (peaks["hbm_gbs"] * 1e9)
+    if tensor_bound:
+        ach = dom["flops"] / dom["s"] / 1e12
+        roof = {"bound": "tensor", "achieved": round(ach, 1), "peak": round(p_fp8_burst, 1), "unit": "TFLOP/s",
+                "frac": round(ach / p_fp8_burst, 3)}
+    else:
+        ach = dom["bytes"] / dom["s"] / 1e9
+        roof = {"bound": "hbm", "achieved": round(ach, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": round(ach / peaks["hbm_gbs"], 3)}
+    roof.update({"traffic": None, "kernel": dom_name, "share": round(dom["s"] / kernel_s, 3),
+                 "peak_source": f"{peaks['source']} (fp8 = {FP8_PER_BF16:g} x bf16 burst)"
+                 if tensor_bound else peaks["source"]})
+
+    # grouped workloads (same method, reported alongside)
+    gtimes = time_problems(grouped, flush, max(3, min(args.steps, 20))) if grouped else []
+    grouped_out = []
+    for p, t in zip(grouped, gtimes):
+        tm = statistics.median(t)
+        c = p.case
+        grouped_out.append({
+            "workload": c.mode + (f" G={c.G} rows={p.case.rows_computed()}" if c.mode == "masked" else
+                                  f" G={c.G} M_total={c.M}"),
+            "N": c.N, "K": c.K, "us": round(tm * 1e6, 2), "tflops": round(p.flops / tm / 1e12, 1),
+            "gbs": round(p.bytes / tm / 1e9, 1),
+            "frac_roof_spec": round(roof_time_s(p.flops, p.bytes, SPEC_FP8_TFLOPS, SPEC_HBM_GBS) / tm, 3),
+            "frac_roof_measured": round(roof_time_s(p.flops, p.bytes, p_fp8_burst, peaks["hbm_gbs"]) / tm, 3),
+            "block_n": p.plan["block_n"]})
+
+    e2e = None
+    if not args.no_e2e:
+        # end to end: pinned host inputs -> device, GEMM, D -> pinned host
+        host = []
+        for p in problems:
+            c = p.case
+            host.append({k: getattr(c, k).cpu().pin_memory() for k in ("A", "sa", "B", "sb")})
+        dev_bufs = [{k: torch.empty_like(getattr(p.case, k)) for k in ("A", "sa", "B", "sb")} for p in problems]
+        d_host = [torch.empty(p.D.shape, dtype=p.D.dtype).pin_memory() for p in problems]
+        h2d = sum(t.numel() * t.element_size() for h in host for t in h.values())
+        d2h = sum(t.numel() * t.element_size() for t in d_host)
+        stream = torch.cuda.current_stream()
+
+        def e2e_step():
+            for p, h, db, dh in zip(problems, host, dev_bufs, d_host):
+                for k in ("A", "sa", "B", "sb"):
+                    db[k].copy_(h[k], non_blocking=True)
+                c = p.case
+                cc = wl.Case(c.mode, c.M, c.N, c.K, c.G, db["A"], db["sa"], c.sa_stride, db["B"], db["sb"])
+                p.run(case=cc)
+                dh.copy_(p.D, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        barrier(world)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e2e_steps = max(1, min(args.steps, 3))
+        e0.record(stream)
+        for _ in range(e2e_steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e2e_s = max_over_ranks(e0.elapsed_time(e1) * 1e-3, world, dev)
+        e2e = {"value": round(aggregate(step_flops * e2e_steps, e2e_s, world), 3), "unit": "TFLOP/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps}
+
+    cpu = cpu_baseline(problems) if (rank == 0 and world == 1 and not args.no_cpu_baseline) else None
+
+    out = {
+        "metric": "FP8 scaled-GEMM TFLOPS per shape; % of B200 FP8 peak or HBM roofline",
+        "value": round(value, 1), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "e4m3 x e4m3 -> f32 accumulate -> bf16",
+        "data": "synthetic (seeded randn inputs quantised to e4m3 with 1x128 / 128x128 FP32 scales)",
+        "config": {"workload": "dense FP8 NT GEMM sweep, 18 shapes: M in {64,128,4096} x (N,K) in "
+                               "{(2112,7168),(24576,1536),(32768,512),(7168,16384),(4096,7168),(7168,2048)}",
+                   "l2": "flushed (512 MiB write) before every GEMM; kernel time from CUDA events",
+                   "parallelism": f"replicas x{world} (weak scaling, no data-path collective)",
+                   "wall_ms_per_step_incl_flush": round(t_wall / args.steps * 1e3, 3)},
+        "per_shape": per_shape,
+        "grouped": grouped_out,
+        "roofline": roof,
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "clocks": clocks,
+        "gpu_launches": len(problems) * args.steps,
+        "peaks": {"fp8_tflops_burst": p_fp8_burst, "hbm_gbs": peaks["hbm_gbs"], "source": peaks["source"],
+                  "spec_fp8_tflops": SPEC_FP8_TFLOPS, "spec_hbm_gbs": SPEC_HBM_GBS},
+    }
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+# ------------------------------------------------------------- reference ----
+
+def run_reference(args, rank, world):
+    """The CPU oracle as the reference arm: each step computes one row per host
+    thread of every shape of the sweep (all N columns), a bounded sample."""
+    if rank != 0:
+        return
+    import oracle
+    threads = oracle.num_threads()
+    cases = [wl.dense_case(m, n, k, seed=0) for (m, n, k) in wl.DENSE_SWEEP]
+    arrays = [(c.A.numpy(), c.sa.numpy(), c.B.numpy(), c.sb.numpy()) for c in cases]
+
+    def step(i):
+        fl = 0.0
+        for c, (A, sa, B, sb) in zip(cases, arrays):
+            rows = oracle_rows_sample(c, threads, salt=i)
+            oracle.gemm_nt(A, sa, c.sa_stride, B, sb, c.M, c.N, c.K, rows=rows, want_d64=False, want_mag=False)
+            fl += 2.0 * len(rows) * c.N * c.K
+        return fl
+
+    for i in range(args.warmup):
+        step(i)
+    t0 = time.perf_counter()
+    fl = sum(step(args.warmup + i) for i in range(args.steps))
+    dt = time.perf_counter() - t0
+    v = fl / dt / 1e12
+    out = {"impl": "reference", "metric": "FP8 scaled-GEMM TFLOPS per shape; % of B200 FP8 peak or HBM roofline",
+           "value": v, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+           "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+           "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+           "config": {"workload": "dense FP8 NT GEMM sweep, 18 shapes: M in {64,128,4096} x (N,K) in "
+                                  "{(2112,7168),(24576,1536),(32768,512),(7168,16384),(4096,7168),(7168,2048)}"},
+           "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                            "sample": f"{threads} full output rows (all N columns) of each of the 18 shapes "
+                                      "per step"},
+           "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
+    ap.add_argument("--no-grouped", action="store_true", help="skip the grouped workloads")
+    ap.add_argument("--shape", default="", help="run one dense shape MxNxK instead of the sweep")
+    args = ap.parse_args(argv)
+    args.warmup = max(args.warmup, 3)  # at least 3 untimed warm-up steps
+    rank, world, local = dist_env()
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    run_ours(args, rank, world, local)
+
+
+if __name__ == "__main__":
+    main()

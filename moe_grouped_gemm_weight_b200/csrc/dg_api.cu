@@ -99,6 +99,23 @@ dg_status make_operand_map(CUtensorMap* tm, const void* base, int K, int rows, i
     return DG_OK;
 }
 
+// bf16 output: dims (N, rows[, groups]), box (32, 32[, 1]) -- one promotion
+// warp's 32 rows x 32 columns -- with 64-byte swizzle; the store clips
+// everything outside the tensor.
+dg_status make_output_map(CUtensorMap* tm, void* base, int N, int rows, int groups, bool three_d) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return fail(DG_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+    cuuint64_t dims[3] = {static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(groups)};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(N) * 2, static_cast<cuuint64_t>(N) * 2 * rows};
+    cuuint32_t box[3] = {32, 32, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, three_d ? 3 : 2, base, dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(DG_ERR_CUDA, "cuTensorMapEncodeTiled (output) failed (CUresult %d)", static_cast<int>(r));
+    return DG_OK;
+}
+
 // ------------------------------------------------------------ planning ----
 
 struct Choice {
@@ -116,32 +133,39 @@ constexpr int max_stages() {
 
 int waves_cost(int tiles, int sms) { return cdiv(tiles, sms); }
 
-// Tile width: the widest N tile (fewer A re-reads, more tensor work per byte
-// of shared memory) unless a narrower one spreads the problem over more SMs
-// -- the point of the "non-aligned block size" optimisation on the DeepGEMM
-// README page (section "非对齐的块大小"), here restricted to N tiles that the
-// promotion warps split into 32-column TMEM loads.
+template <int BN>
+constexpr int smem_for() {
+    return dg::smem_bytes<BN, max_stages<BN>()>();
+}
+
+// Tile width.  Each 128-wide K block costs a tile max(MMA time, operand
+// streaming time): the tensor core's time grows with BN, while the bytes
+// moved into shared memory are 16 KiB of A plus BN*128 B of B.  Relative
+// units: MMA = BN, streaming = 0.75*(128 + BN).  The problem takes
+// ceil(tiles / SMs) such tile times.  Narrower tiles win when they put more
+// SMs to work -- the point of the "non-aligned block size" optimisation on
+// the DeepGEMM README page (section "非对齐的块大小"); here BN stays a
+// multiple of 64 so that the two promotion warpgroups split it into 32-column
+// TMEM loads.
 Choice choose(int m_blocks, int N, int num_sms) {
-    const int cands[2] = {128, 64};
+    const int cands[3] = {256, 128, 64};
     Choice best{128, max_stages<128>()};
-    long best_cost = -1;
+    double best_cost = -1.0;
     for (int bn : cands) {
         const int tiles = m_blocks * cdiv(N, bn);
-        // Cost model: waves of tiles times the per-tile time, taken as
-        // proportional to the tile width (both operands stream per K block).
-        const long cost = static_cast<long>(waves_cost(tiles, num_sms)) * (bn + 128);
-        if (best_cost < 0 || cost < best_cost) {
+        const double t_kb = bn > 0.75 * (128 + bn) ? bn : 0.75 * (128 + bn);
+        const double cost = static_cast<double>(waves_cost(tiles, num_sms)) * t_kb;
+        if (best_cost < 0 || cost < best_cost - 1e-9) {
             best_cost = cost;
             best.bn = bn;
         }
     }
-    best.stages = best.bn == 128 ? max_stages<128>() : max_stages<64>();
+    best.stages = best.bn == 256 ? max_stages<256>() : best.bn == 128 ? max_stages<128>() : max_stages<64>();
     return best;
 }
 
 int plan_smem(const Choice& c) {
-    return c.bn == 128 ? dg::smem_bytes<128, 8>() - (8 - c.stages) * (dg::kTileABytes + 128 * dg::kBK)
-                       : dg::smem_bytes<64, 8>() - (8 - c.stages) * (dg::kTileABytes + 64 * dg::kBK);
+    return c.bn == 256 ? smem_for<256>() : c.bn == 128 ? smem_for<128>() : smem_for<64>();
 }
 
 dg_status check_sizes(int mode, int rows, int N, int K, int G) {
@@ -182,8 +206,8 @@ dg_status plan(int mode, int rows, int N, int K, int G, int num_sms, dg_plan* ou
 // ------------------------------------------------------------ launch ----
 
 template <int BN, int STAGES, int MODE>
-dg_status launch_one(const dg::Params& p, const CUtensorMap& ta, const CUtensorMap& tb, int grid,
-                     cudaStream_t stream) {
+dg_status launch_one(const dg::Params& p, const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& td,
+                     int grid, cudaStream_t stream) {
     constexpr int smem = dg::smem_bytes<BN, STAGES>();
     static_assert(smem <= 227 * 1024, "shared memory budget exceeded");
     auto kern = dg::fp8_gemm_kernel<BN, STAGES, MODE>;
@@ -195,7 +219,7 @@ dg_status launch_one(const dg::Params& p, const CUtensorMap& ta, const CUtensorM
             return fail(DG_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(cudaGetLastError()));
         attr_set[dev].store(1);
     }
-    kern<<<grid, dg::kThreads, smem, stream>>>(p, ta, tb);
+    kern<<<grid, dg::kThreads, smem, stream>>>(p, ta, tb, td);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return fail(DG_ERR_CUDA, "kernel launch failed: %s", cudaGetErrorString(e));
     return ok();
@@ -203,13 +227,13 @@ dg_status launch_one(const dg::Params& p, const CUtensorMap& ta, const CUtensorM
 
 template <int MODE>
 dg_status dispatch(const dg_plan& pl, const dg::Params& p, const CUtensorMap& ta, const CUtensorMap& tb,
-                   cudaStream_t stream) {
-    if (pl.block_n == 128) {
-        constexpr int S = max_stages<128>();
-        return launch_one<128, S, MODE>(p, ta, tb, pl.grid, stream);
+                   const CUtensorMap& td, cudaStream_t stream) {
+    switch (pl.block_n) {
+        case 256: return launch_one<256, max_stages<256>(), MODE>(p, ta, tb, td, pl.grid, stream);
+        case 128: return launch_one<128, max_stages<128>(), MODE>(p, ta, tb, td, pl.grid, stream);
+        case 64: return launch_one<64, max_stages<64>(), MODE>(p, ta, tb, td, pl.grid, stream);
+        default: return fail(DG_ERR_UNSUPPORTED, "no kernel for block_n=%d", pl.block_n);
     }
-    constexpr int S = max_stages<64>();
-    return launch_one<64, S, MODE>(p, ta, tb, pl.grid, stream);
 }
 
 int effective_sms() {
@@ -245,6 +269,7 @@ dg::Params make_params(uint16_t* D, const float* sa, int sa_stride, const float*
     p.n_blocks = pl.n_blocks;
     p.m_blocks = pl.m_blocks;
     p.raster = 8;
+    p.b_stream = 0;
     return p;
 }
 
@@ -265,8 +290,11 @@ dg_status dg_fp8_gemm_nt(uint16_t* D, const uint8_t* A, const float* sa, int sa_
     CUtensorMap ta, tb;
     if ((s = make_operand_map(&ta, A, K, M, 1, dg::kBM, false)) != DG_OK) return s;
     if ((s = make_operand_map(&tb, B, K, N, 1, pl.block_n, true)) != DG_OK) return s;
+    CUtensorMap td;
+    if ((s = make_output_map(&td, D, N, M, 1, false)) != DG_OK) return s;
     dg::Params p = make_params(D, sa, sa_stride, sb, M, N, K, 1, pl);
-    return dispatch<dg::kDense>(pl, p, ta, tb, static_cast<cudaStream_t>(stream));
+    p.b_stream = pl.m_blocks == 1;
+    return dispatch<dg::kDense>(pl, p, ta, tb, td, static_cast<cudaStream_t>(stream));
 }
 
 dg_status dg_grouped_contiguous_nt(uint16_t* D, const uint8_t* A, const float* sa, int sa_stride, const uint8_t* B,
@@ -284,9 +312,11 @@ dg_status dg_grouped_contiguous_nt(uint16_t* D, const uint8_t* A, const float* s
     CUtensorMap ta, tb;
     if ((s = make_operand_map(&ta, A, K, M_total, 1, dg::kBM, false)) != DG_OK) return s;
     if ((s = make_operand_map(&tb, B, K, N, G, pl.block_n, true)) != DG_OK) return s;
+    CUtensorMap td;
+    if ((s = make_output_map(&td, D, N, M_total, 1, false)) != DG_OK) return s;
     dg::Params p = make_params(D, sa, sa_stride, sb, M_total, N, K, G, pl);
     p.m_indices = m_indices;
-    return dispatch<dg::kContiguous>(pl, p, ta, tb, static_cast<cudaStream_t>(stream));
+    return dispatch<dg::kContiguous>(pl, p, ta, tb, td, static_cast<cudaStream_t>(stream));
 }
 
 dg_status dg_grouped_masked_nt(uint16_t* D, const uint8_t* A, const float* sa, int sa_stride, const uint8_t* B,
@@ -305,9 +335,12 @@ dg_status dg_grouped_masked_nt(uint16_t* D, const uint8_t* A, const float* sa, i
     CUtensorMap ta, tb;
     if ((s = make_operand_map(&ta, A, K, M_max, G, dg::kBM, true)) != DG_OK) return s;
     if ((s = make_operand_map(&tb, B, K, N, G, pl.block_n, true)) != DG_OK) return s;
+    CUtensorMap td;
+    if ((s = make_output_map(&td, D, N, M_max, G, true)) != DG_OK) return s;
     dg::Params p = make_params(D, sa, sa_stride, sb, M_max, N, K, G, pl);
     p.masked_m = masked_m;
-    return dispatch<dg::kMasked>(pl, p, ta, tb, static_cast<cudaStream_t>(stream));
+    p.b_stream = M_max <= dg::kBM;
+    return dispatch<dg::kMasked>(pl, p, ta, tb, td, static_cast<cudaStream_t>(stream));
 }
 
 void dg_set_num_sms(int n) { g_num_sms_cap.store(n > 0 ? n : 0); }

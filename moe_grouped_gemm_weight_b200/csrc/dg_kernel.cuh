@@ -2,19 +2,24 @@
 // block-scaled NT GEMM (dense, grouped-contiguous and grouped-masked forms).
 //
 // Per output tile of 128 x BN:
-//   * warp 0 (producer): TMA-loads, for every 128-wide K block kb, the A tile
-//     [128 rows x 128 K] and the B tile [BN rows x 128 K] (128-byte swizzle)
-//     into a STAGES-deep shared-memory ring.
+//   * warp 0 (operand producer): TMA-loads, for every 128-wide K block kb,
+//     the A tile [128 rows x 128 K] and the B tile [BN rows x 128 K]
+//     (128-byte swizzle) into a STAGES-deep shared-memory ring.
 //   * warp 1 (MMA): issues four tcgen05.mma kind::f8f6f4 (K = 32 each) that
 //     write P_kb = A_kb . B_kb^T into a FRESH TMEM buffer (one of NBUF), then
 //     commits to the ring's "empty" barrier and the buffer's "full" barrier.
-//   * warps 4..11 (promotion + epilogue): pull P_kb out of TMEM with
-//     tcgen05.ld, release the buffer, and accumulate
+//   * warp 2 (scale producer): copies sa[m0..m0+127, kb] and the one or two
+//     sb[n/128, kb] the tile needs into a 16-deep shared-memory scale ring,
+//     running ahead of the promotion so that no global-memory latency sits on
+//     its critical path.
+//   * warps 4..11 (promotion + epilogue, two warpgroups splitting the tile's
+//     columns): pull P_kb out of TMEM with tcgen05.ld, release the buffer,
+//     and accumulate
 //         acc[m,n] += (sa[m,kb] * sb[n/128,kb]) * P_kb[m,n]
-//     in FP32 registers -- the two-level accumulation with promotion interval
-//     128 described on the page "Deepseek DeepGEMM 技术原理的深入分析" (section
-//     "技术背景与核心原理").  After the last kb they round to bf16 and store
-//     the valid rows and columns.
+//     in FP32 registers with packed FP32x2 FMAs -- the two-level accumulation
+//     with promotion interval 128 described on the page "Deepseek DeepGEMM
+//     技术原理的深入分析" (section "技术背景与核心原理").  After the last kb
+//     they round to bf16 and store the valid rows and columns.
 // TMEM buffers let the tensor core run up to NBUF-1 blocks ahead of the
 // promotion, and the next tile's MMAs overlap the previous tile's epilogue.
 // Tiles are handed out round-robin over a rasterised order (groups of
@@ -37,6 +42,9 @@ constexpr int kFirstEpiWarp = 4;         // warps 4..11: promotion/epilogue
 constexpr int kEpiWarps = 8;
 constexpr int kTileABytes = kBM * kBK;   // 16 KiB of e4m3
 constexpr int kMaxMaskedGroups = 1024;   // masked mode: prefix table in smem
+constexpr int kScaleSlots = 16;          // depth of the scale ring
+constexpr int kScaleSlotFloats = kBM + 4;  // sa for 128 rows + up to 4 sb values
+constexpr int kStageOutBytes = 32 * 32 * 2;  // per promotion warp: 32 rows x 32 bf16 columns
 
 struct Params {
     uint16_t* D;
@@ -52,6 +60,7 @@ struct Params {
     int n_blocks;   // ceil(N / BN)
     int m_blocks;   // dense/contiguous: ceil(M / 128); masked: unused (device prefix)
     int raster;     // m-blocks per raster group
+    int b_stream;   // 1: B is read once (evict-first in L2), 0: B is reused
 };
 
 template <int BN>
@@ -60,22 +69,26 @@ struct Cfg {
     static constexpr int kTileBBytes = BN * kBK;
     static constexpr int kNBuf = (BN <= 128) ? 4 : 2;
     static constexpr int kTmemCols = (kNBuf * BN <= 256) ? 256 : 512;
-    static constexpr int kColsPerWarp = BN / 2;       // two warpgroups split the columns
+    static constexpr int kColsPerWarp = BN / 2;        // two warpgroups split the columns
     static constexpr int kChunks = kColsPerWarp / 32;  // tcgen05.ld 32x32b.x32 chunks
+    static constexpr int kBatch = kChunks < 2 ? kChunks : 2;  // chunks loaded per wait
+    static constexpr bool kSplitRegs = BN > 128;       // needs setmaxnreg rebalancing
     static_assert(kNBuf * BN <= kTmemCols, "TMEM buffers overflow the allocation");
+    static_assert(kChunks % kBatch == 0, "chunk batching");
 };
 
 template <int BN, int STAGES>
 constexpr int smem_bytes() {
-    // 1 KiB alignment slack + operand ring + barriers / bookkeeping + masked prefix table.
-    return 1024 + STAGES * (kTileABytes + Cfg<BN>::kTileBBytes) + 256 + 4 * (kMaxMaskedGroups + 1);
+    // 1 KiB alignment slack + operand ring + output staging + barriers and
+    // bookkeeping (512 B) + scale ring + masked prefix table.
+    return 1024 + STAGES * (kTileABytes + Cfg<BN>::kTileBBytes) + kEpiWarps * kStageOutBytes + 512 +
+           kScaleSlots * kScaleSlotFloats * 4 + 4 * (kMaxMaskedGroups + 1);
 }
 
 struct Tile {
     int g;        // group
-    int a_row;    // A row coordinate (dense/contiguous: global row; masked: row inside group)
+    int m0;       // first output row (dense/contiguous: global; masked: inside group g)
     int n0;       // first output column
-    int m0;       // first output row (dense/contiguous: global; masked: inside group)
     bool valid;
 };
 
@@ -100,9 +113,9 @@ __device__ __forceinline__ Tile decode_tile(const Params& p, int t, int m_blocks
     tl.valid = true;
     if (MODE == kDense) {
         tl.g = 0;
-        tl.m0 = tl.a_row = mb * kBM;
+        tl.m0 = mb * kBM;
     } else if (MODE == kContiguous) {
-        tl.m0 = tl.a_row = mb * kBM;
+        tl.m0 = mb * kBM;
         const int g = __ldg(p.m_indices + tl.m0);
         // A tile whose first row is padding holds only padding (segments are
         // aligned to 128 rows and padded at their end); out-of-range group
@@ -117,7 +130,7 @@ __device__ __forceinline__ Tile decode_tile(const Params& p, int t, int m_blocks
             if (mb_prefix[mid] <= mb) lo = mid; else hi = mid - 1;
         }
         tl.g = lo;
-        tl.m0 = tl.a_row = (mb - mb_prefix[lo]) * kBM;
+        tl.m0 = (mb - mb_prefix[lo]) * kBM;
     }
     return tl;
 }
@@ -125,7 +138,7 @@ __device__ __forceinline__ Tile decode_tile(const Params& p, int t, int m_blocks
 template <int BN, int STAGES, int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
 fp8_gemm_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtensorMap tmA,
-                const __grid_constant__ CUtensorMap tmB) {
+                const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmD) {
     using C = Cfg<BN>;
     constexpr int kNBuf = C::kNBuf;
 
@@ -133,14 +146,18 @@ fp8_gemm_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtens
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* sA = smem;
     uint8_t* sB = sA + STAGES * kTileABytes;
-    uint64_t* full = reinterpret_cast<uint64_t*>(sB + STAGES * C::kTileBBytes);
+    uint8_t* sOut = sB + STAGES * C::kTileBBytes;  // 1 KiB aligned, kStageOutBytes per promotion warp
+    uint64_t* full = reinterpret_cast<uint64_t*>(sOut + kEpiWarps * kStageOutBytes);
     uint64_t* empty = full + STAGES;
     uint64_t* tfull = empty + STAGES;
     uint64_t* tempty = tfull + kNBuf;
-    uint64_t* done = tempty + kNBuf;
+    uint64_t* sfull = tempty + kNBuf;
+    uint64_t* sempty = sfull + kScaleSlots;
+    uint64_t* done = sempty + kScaleSlots;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-    int* mb_prefix = const_cast<int*>(reinterpret_cast<volatile int*>(abort_flag + 1));
+    float* sring = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(full) + 512);
+    int* mb_prefix = reinterpret_cast<int*>(sring + kScaleSlots * kScaleSlotFloats);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -154,6 +171,10 @@ fp8_gemm_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtens
             mbar_init(tfull + b, 1);
             mbar_init(tempty + b, kEpiWarps);
         }
+        for (int s = 0; s < kScaleSlots; ++s) {
+            mbar_init(sfull + s, 32);
+            mbar_init(sempty + s, kEpiWarps);
+        }
         mbar_init(done, 1);
         *abort_flag = 0;
         fence_mbar_init();
@@ -161,6 +182,7 @@ fp8_gemm_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtens
     if (warp == 0 && lane == 0) {
         prefetch_tmap(&tmA);
         prefetch_tmap(&tmB);
+        prefetch_tmap(&tmD);
     }
     if (warp == 1) {
         tmem_alloc(tmem_slot, C::kTmemCols);
@@ -204,10 +226,15 @@ fp8_gemm_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtens
     const int tiles = m_blocks * p.n_blocks;
     const int nkb = p.nkb;
 
+    // Register budget: the producer / MMA / scale warps need few registers,
+    // the promotion warps hold BN/2 FP32 accumulators each.  Each branch sets
+    // its own budget so that the compiler allocates every role against it.
+    if (warp < kFirstEpiWarp) {
+    if (C::kSplitRegs) regs_dec<56>();
     if (warp == 0) {
         // ------------------------------------------------------ producer ----
         const uint64_t pol_a = l2_policy_evict_last();
-        const uint64_t pol_b = l2_policy_evict_last();
+        const uint64_t pol_b = p.b_stream ? l2_policy_evict_first() : l2_policy_evict_last();
         int stage = 0;
         uint32_t phase = 0;
         int fills = 0;
@@ -220,9 +247,9 @@ fp8_gemm_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtens
                 if (lane == 0) {
                     mbar_arrive_expect_tx(full + stage, kTileABytes + C::kTileBBytes);
                     if (MODE == kMasked)
-                        tma_load_3d(sA + stage * kTileABytes, &tmA, full + stage, kb * kBK, tl.a_row, tl.g, pol_a);
+                        tma_load_3d(sA + stage * kTileABytes, &tmA, full + stage, kb * kBK, tl.m0, tl.g, pol_a);
                     else
-                        tma_load_2d(sA + stage * kTileABytes, &tmA, full + stage, kb * kBK, tl.a_row, pol_a);
+                        tma_load_2d(sA + stage * kTileABytes, &tmA, full + stage, kb * kBK, tl.m0, pol_a);
                     tma_load_3d(sB + stage * C::kTileBBytes, &tmB, full + stage, kb * kBK, tl.n0, tl.g, pol_b);
                 }
                 __syncwarp();
@@ -273,105 +300,186 @@ fp8_gemm_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtens
             mbar_wait_drain(done, 0);
         }
         __syncwarp();
-    } else if (warp >= kFirstEpiWarp) {
+    } else if (warp == 2) {
+        // ------------------------------------------------ scale producer ----
+        int slot = 0;
+        uint32_t sphase = 0;
+        bool ok = true;
+        const int row_limit = p.M;  // rows of sa that exist (dense M, M_total or M_max)
+        for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
+            const Tile tl = decode_tile<BN, MODE>(p, t, m_blocks, mb_prefix);
+            if (!tl.valid) continue;
+            const float* sa_base = p.sa + (MODE == kMasked ? static_cast<int64_t>(tl.g) * nkb * p.sa_stride : 0);
+            const float* sb_g = p.sb + static_cast<int64_t>(tl.g) * p.nbn * nkb;
+            const int nb_first = tl.n0 / 128;
+            const int r4 = tl.m0 + lane * 4;
+            for (int kb = 0; kb < nkb; ++kb) {
+                if (!mbar_wait(sempty + slot, sphase ^ 1u, abort_flag)) { ok = false; break; }
+                const float* src = sa_base + static_cast<int64_t>(kb) * p.sa_stride + r4;
+                float4 v;
+                if (r4 + 3 < row_limit) {
+                    v = ld_nc_f4(src);
+                } else {
+                    v.x = r4 + 0 < row_limit ? __ldg(src + 0) : 0.f;
+                    v.y = r4 + 1 < row_limit ? __ldg(src + 1) : 0.f;
+                    v.z = r4 + 2 < row_limit ? __ldg(src + 2) : 0.f;
+                    v.w = r4 + 3 < row_limit ? __ldg(src + 3) : 0.f;
+                }
+                float* dst = sring + slot * kScaleSlotFloats;
+                *reinterpret_cast<float4*>(dst + lane * 4) = v;
+                if (lane < 4) {
+                    const int nb = min(nb_first + lane, p.nbn - 1);
+                    dst[kBM + lane] = __ldg(sb_g + static_cast<int64_t>(nb) * nkb + kb);
+                }
+                mbar_arrive(sfull + slot);
+                if (++slot == kScaleSlots) { slot = 0; sphase ^= 1u; }
+            }
+        }
+    }
+    } else {
         // ------------------------------------------ promotion + epilogue ----
+        if (C::kSplitRegs) regs_inc<224>();
         const int ew = warp - kFirstEpiWarp;
         const int half = ew >> 2;                 // which half of the tile's columns
         const int quarter = warp & 3;             // TMEM lane quarter this warp may access
         const int r = quarter * 32 + lane;        // row inside the tile
         const int col0 = half * C::kColsPerWarp;  // first column inside the tile
         const uint32_t t_lane = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16);
-        int buf = 0;
-        uint32_t bphase = 0;
+        int buf = 0, slot = 0;
+        uint32_t bphase = 0, sphase = 0;
         bool ok = true;
         for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
             const Tile tl = decode_tile<BN, MODE>(p, t, m_blocks, mb_prefix);
             if (!tl.valid) continue;
             const int g = tl.g;
-            // Row validity and the row's output / scale addresses.
+            // Row validity and the row's output address.
             const int row = tl.m0 + r;
             bool row_ok;
             int64_t d_row;
-            const float* sa_row;
             if (MODE == kMasked) {
                 const int mm = min(max(__ldg(p.masked_m + g), 0), p.M);
                 row_ok = row < mm;
                 d_row = static_cast<int64_t>(g) * p.M + row;
-                sa_row = p.sa + static_cast<int64_t>(g) * nkb * p.sa_stride + row;
             } else if (MODE == kContiguous) {
                 const int gi = __ldg(p.m_indices + row);
                 row_ok = (gi == g);
                 if (gi != g && gi != -1) atomicOr(&g_dg_error, 2u);
                 d_row = row;
-                sa_row = p.sa + row;
             } else {
                 row_ok = row < p.M;
                 d_row = row;
-                sa_row = p.sa + row;
             }
-            const float* sb_g = p.sb + static_cast<int64_t>(g) * p.nbn * nkb;
-            int nb_idx[C::kChunks];
+            // Which of the scale ring's sb values each 32-column chunk uses.
+            int sb_sel[C::kChunks];
 #pragma unroll
-            for (int c = 0; c < C::kChunks; ++c)
-                nb_idx[c] = min((tl.n0 + col0 + c * 32) / 128, p.nbn - 1);
+            for (int c = 0; c < C::kChunks; ++c) sb_sel[c] = (tl.n0 + col0 + c * 32) / 128 - tl.n0 / 128;
 
-            float acc[C::kColsPerWarp];
+            float2 acc[C::kColsPerWarp / 2];
 #pragma unroll
-            for (int j = 0; j < C::kColsPerWarp; ++j) acc[j] = 0.f;
+            for (int j = 0; j < C::kColsPerWarp / 2; ++j) acc[j] = make_float2(0.f, 0.f);
 
             for (int kb = 0; kb < nkb; ++kb) {
-                const float s_a = row_ok ? __ldg(sa_row + static_cast<int64_t>(kb) * p.sa_stride) : 0.f;
-                float s[C::kChunks];
+                if (!mbar_wait(sfull + slot, sphase, abort_flag)) { ok = false; break; }
+                const float* sc = sring + slot * kScaleSlotFloats;
+                const float s_a = sc[r];
+                float2 s2[C::kChunks];
 #pragma unroll
-                for (int c = 0; c < C::kChunks; ++c) s[c] = s_a * __ldg(sb_g + nb_idx[c] * nkb + kb);
+                for (int c = 0; c < C::kChunks; ++c) {
+                    const float s = s_a * sc[kBM + sb_sel[c]];
+                    s2[c] = make_float2(s, s);
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(sempty + slot);
+                if (++slot == kScaleSlots) { slot = 0; sphase ^= 1u; }
 
                 if (!mbar_wait(tfull + buf, bphase, abort_flag)) { ok = false; break; }
                 tc_fence_after();
-                uint32_t v[C::kChunks][32];
 #pragma unroll
-                for (int c = 0; c < C::kChunks; ++c)
-                    tmem_ld_32x32b_x32(t_lane + static_cast<uint32_t>(buf * BN + col0 + c * 32), v[c]);
-                tmem_ld_wait();
+                for (int cb = 0; cb < C::kChunks; cb += C::kBatch) {
+                    uint32_t v[C::kBatch][32];
 #pragma unroll
-                for (int c = 0; c < C::kChunks; ++c) reg_fence(v[c]);
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(tempty + buf);
+                    for (int c = 0; c < C::kBatch; ++c)
+                        tmem_ld_32x32b_x32(t_lane + static_cast<uint32_t>(buf * BN + col0 + (cb + c) * 32), v[c]);
+                    tmem_ld_wait();
 #pragma unroll
-                for (int c = 0; c < C::kChunks; ++c)
+                    for (int c = 0; c < C::kBatch; ++c) reg_fence(v[c]);
+                    if (cb + C::kBatch == C::kChunks) {
+                        // Last TMEM read of this buffer: hand it back to the MMA warp.
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(tempty + buf);
+                    }
 #pragma unroll
-                    for (int j = 0; j < 32; ++j)
-                        acc[c * 32 + j] = fmaf(__uint_as_float(v[c][j]), s[c], acc[c * 32 + j]);
+                    for (int c = 0; c < C::kBatch; ++c)
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) {
+                            const float2 pv = make_float2(__uint_as_float(v[c][2 * j]), __uint_as_float(v[c][2 * j + 1]));
+                            acc[(cb + c) * 16 + j] = __ffma2_rn(pv, s2[cb + c], acc[(cb + c) * 16 + j]);
+                        }
+                }
                 if (++buf == kNBuf) { buf = 0; bphase ^= 1u; }
             }
             if (!ok) break;
 
-            // Epilogue: bf16 round-to-nearest-even, 16-byte stores of the valid
-            // part of this row (N % 8 == 0, so 8-column groups are all-or-none).
-            if (row_ok) {
-                uint16_t* drow = p.D + d_row * p.N;
+            // Epilogue: bf16 round-to-nearest-even.  When every row of this
+            // warp may be written (valid, or outside D where the TMA store
+            // clips it), the warp stages 32 rows x 32 columns at a time in
+            // shared memory (64-byte swizzle: 16-byte chunk q of row r sits at
+            // r*64 + 16*(q ^ ((r >> 1) & 3)), conflict-free for the warp) and
+            // one lane issues a TMA store; the copy drains while the warp
+            // moves on.  Warps holding rows that must stay untouched (padding
+            // rows, rows past masked_m) store their valid rows directly.
+            const bool clip_ok = row_ok || MODE == kDense || (MODE == kMasked && row >= p.M);
+            if (__all_sync(0xffffffffu, clip_ok)) {
+                const uint32_t stg = smem_u32(sOut + ew * kStageOutBytes);
 #pragma unroll
-                for (int c = 0; c < C::kChunks; ++c) {
+                for (int pc = 0; pc < C::kColsPerWarp / 32; ++pc) {
+                    if (lane == 0) bulk_wait_read<0>();  // previous store has read the buffer
+                    __syncwarp();
 #pragma unroll
                     for (int q = 0; q < 4; ++q) {
-                        const int col = tl.n0 + col0 + c * 32 + q * 8;
-                        if (col < p.N) {
-                            uint4 pk;
-                            const float* a8 = acc + c * 32 + q * 8;
-                            __nv_bfloat162 h0 = __floats2bfloat162_rn(a8[0], a8[1]);
-                            __nv_bfloat162 h1 = __floats2bfloat162_rn(a8[2], a8[3]);
-                            __nv_bfloat162 h2 = __floats2bfloat162_rn(a8[4], a8[5]);
-                            __nv_bfloat162 h3 = __floats2bfloat162_rn(a8[6], a8[7]);
-                            pk.x = *reinterpret_cast<uint32_t*>(&h0);
-                            pk.y = *reinterpret_cast<uint32_t*>(&h1);
-                            pk.z = *reinterpret_cast<uint32_t*>(&h2);
-                            pk.w = *reinterpret_cast<uint32_t*>(&h3);
-                            *reinterpret_cast<uint4*>(drow + col) = pk;
-                        }
+                        __nv_bfloat162 h0 = __float22bfloat162_rn(acc[pc * 16 + q * 4 + 0]);
+                        __nv_bfloat162 h1 = __float22bfloat162_rn(acc[pc * 16 + q * 4 + 1]);
+                        __nv_bfloat162 h2 = __float22bfloat162_rn(acc[pc * 16 + q * 4 + 2]);
+                        __nv_bfloat162 h3 = __float22bfloat162_rn(acc[pc * 16 + q * 4 + 3]);
+                        const uint32_t off = lane * 64 + ((q ^ ((lane >> 1) & 3)) << 4);
+                        st_shared_v4(stg + off, *reinterpret_cast<uint32_t*>(&h0), *reinterpret_cast<uint32_t*>(&h1),
+                                     *reinterpret_cast<uint32_t*>(&h2), *reinterpret_cast<uint32_t*>(&h3));
+                    }
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    const int x = tl.n0 + col0 + pc * 32;
+                    if (lane == 0 && x < p.N) {
+                        if (MODE == kMasked)
+                            tma_store_3d(&tmD, sOut + ew * kStageOutBytes, x, tl.m0 + quarter * 32, g);
+                        else
+                            tma_store_2d(&tmD, sOut + ew * kStageOutBytes, x, tl.m0 + quarter * 32);
+                        bulk_commit();
+                    }
+                }
+            } else if (row_ok) {
+                uint16_t* drow = p.D + d_row * p.N;
+#pragma unroll
+                for (int q = 0; q < C::kColsPerWarp / 8; ++q) {
+                    const int col = tl.n0 + col0 + q * 8;
+                    if (col < p.N) {
+                        uint4 pk;
+                        __nv_bfloat162 h0 = __float22bfloat162_rn(acc[q * 4 + 0]);
+                        __nv_bfloat162 h1 = __float22bfloat162_rn(acc[q * 4 + 1]);
+                        __nv_bfloat162 h2 = __float22bfloat162_rn(acc[q * 4 + 2]);
+                        __nv_bfloat162 h3 = __float22bfloat162_rn(acc[q * 4 + 3]);
+                        pk.x = *reinterpret_cast<uint32_t*>(&h0);
+                        pk.y = *reinterpret_cast<uint32_t*>(&h1);
+                        pk.z = *reinterpret_cast<uint32_t*>(&h2);
+                        pk.w = *reinterpret_cast<uint32_t*>(&h3);
+                        *reinterpret_cast<uint4*>(drow + col) = pk;
                     }
                 }
             }
         }
+        // Every TMA store of this warp must have completed before the CTA exits.
+        if (lane == 0) bulk_wait<0>();
+        __syncwarp();
     }
 
     tc_fence_before();
