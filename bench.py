@@ -165,7 +165,10 @@ class Problem:
         self.bytes = c.bytes()
         mode = {"dense": 0, "contiguous": 1, "masked": 2}[c.mode]
         self.plan = dg.dg_make_plan(mode, c.M, c.N, c.K, c.G, dg.dg_get_num_sms())
-        self.kernel = f"fp8_gemm_kernel<BN={self.plan['block_n']},STAGES={self.plan['stages']},{c.mode}>"
+        pl = self.plan
+        # Names of the C++ template instances the call launches.
+        self.kernel = (f"fp8_gemm_swapab_kernel<{pl['block_m']}, {mode}>" if pl["swap_ab"] else
+                       f"fp8_gemm_kernel<{pl['block_n']}, {pl['stages']}, {mode}>")
 
     def run(self, case=None, D=None):
         c = case or self.case
@@ -176,6 +179,33 @@ class Problem:
             self.dg.dg_grouped_contiguous_nt(D, c.A, c.sa, c.sa_stride, c.B, c.sb, c.m_indices)
         else:
             self.dg.dg_grouped_masked_nt(D, c.A, c.sa, c.sa_stride, c.B, c.sb, c.masked_m)
+
+
+def kernel_source_sha() -> str:
+    import glob
+    import hashlib
+    h = hashlib.sha256()
+    for f in sorted(glob.glob(os.path.join(ROOT, "moe_grouped_gemm_weight_b200", "csrc", "*"))):
+        h.update(os.path.basename(f).encode())
+        with open(f, "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel: str):
+    """DRAM bytes per launch recorded by ncu under profiles/ for `kernel`, if the
+    kernel sources have not changed since the capture (else None)."""
+    import glob
+    for path in glob.glob(os.path.join(ROOT, "profiles", "dram_traffic_*.txt")):
+        kv = {}
+        with open(path) as f:
+            for line in f:
+                if "=" in line and not line.startswith("#") and " " not in line.split("=")[0].strip():
+                    k, v = line.split("=", 1)
+                    kv[k.strip()] = v.strip()
+        if kv.get("kernel") == kernel and kv.get("kernel_source_sha") == kernel_source_sha():
+            return int(kv["traffic_per_launch"]), os.path.relpath(path, ROOT)
+    return None, None
 
 
 def roof_time_s(flops, byts, tflops, gbs):
@@ -308,7 +338,10 @@ def run_ours(args, rank, world, local):
         ach = dom["bytes"] / dom["s"] / 1e9
         roof = {"bound": "hbm", "achieved": round(ach, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": round(ach / peaks["hbm_gbs"], 3)}
-    roof.update({"traffic": None, "kernel": dom_name, "share": round(dom["s"] / kernel_s, 3),
+    traffic, traffic_src = recorded_traffic(dom_name)
+    roof.update({"traffic": traffic, "traffic_source": traffic_src,
+                 "algorithmic_bytes_per_launch": int(dom["bytes"] / dom["launches"]),
+                 "kernel": dom_name, "share": round(dom["s"] / kernel_s, 3),
                  "peak_source": f"{peaks['source']} (fp8 = {FP8_PER_BF16:g} x bf16 burst)"
                  if tensor_bound else peaks["source"]})
 

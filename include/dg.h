@@ -130,6 +130,13 @@ DG_API int dg_get_tma_aligned_size(int x, int elem_bytes);
  * in *code.  Synchronises the device first; meant for tests and debugging. */
 DG_API dg_status dg_get_device_error(int* code);
 
+/* Failure-detection self-test: launches one CTA that waits on an mbarrier
+ * nothing ever completes.  The kernels' bounded wait gives up after about one
+ * second, sets DG_DEVERR_TIMEOUT in the device error word and returns, so the
+ * context stays usable.  Enqueued on `stream`; read the outcome with
+ * dg_get_device_error().  Diagnostic only (no counterpart on the pages). */
+DG_API dg_status dg_selftest_bounded_wait(void* stream);
+
 /* Static text for a status code. */
 DG_API const char* dg_status_string(dg_status s);
 /* Text describing the last failing call on this host thread ("" if none). */
@@ -141,14 +148,16 @@ DG_API const char* dg_last_error_message(void);
  * (contiguous) or M_max (masked).  Returns DG_ERR_INVALID_ARG for bad sizes.
  */
 typedef struct dg_plan {
-    int block_m;      /* output rows per tile (tcgen05 M)                       */
-    int block_n;      /* output columns per tile (tcgen05 N)                     */
+    int block_m;      /* output rows per tile                                    */
+    int block_n;      /* output columns per tile                                 */
     int stages;       /* depth of the shared-memory operand ring                 */
-    int m_blocks;     /* tiles along M (masked: worst case, G*ceil(M_max/BM))    */
+    int m_blocks;     /* tiles along M (masked: worst case, G*ceil(M_max/block_m)) */
     int n_blocks;     /* tiles along N                                           */
     int tiles;        /* m_blocks * n_blocks                                     */
-    int grid;         /* persistent CTAs launched                                */
+    int grid;         /* CTAs launched                                           */
     int smem_bytes;   /* dynamic shared memory per CTA                           */
+    int swap_ab;      /* 1: few-row kernel (weights on the MMA's 128-row side)   */
+    int split_k;      /* CTAs (one thread-block cluster) sharing each tile's K   */
 } dg_plan;
 
 DG_API dg_status dg_make_plan(int mode, int rows, int N, int K, int G, int num_sms, dg_plan* out);

@@ -38,7 +38,8 @@ class DGError(RuntimeError):
 
 class Plan(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int) for n in
-                ("block_m", "block_n", "stages", "m_blocks", "n_blocks", "tiles", "grid", "smem_bytes")]
+                ("block_m", "block_n", "stages", "m_blocks", "n_blocks", "tiles", "grid", "smem_bytes",
+                 "swap_ab", "split_k")]
 
     def as_dict(self) -> dict:
         return {n: getattr(self, n) for n, _ in self._fields_}
@@ -73,6 +74,8 @@ def lib() -> ctypes.CDLL:
             L.dg_status_string.argtypes = [I]
             L.dg_last_error_message.restype = ctypes.c_char_p
             L.dg_last_error_message.argtypes = []
+            L.dg_selftest_bounded_wait.restype = I
+            L.dg_selftest_bounded_wait.argtypes = [P]
             L.dg_make_plan.restype = I
             L.dg_make_plan.argtypes = [I, I, I, I, I, I, ctypes.POINTER(Plan)]
             _lib = L
@@ -150,6 +153,11 @@ def dg_make_plan(mode: int, rows: int, N: int, K: int, G: int, num_sms: int) -> 
     _check("dg_make_plan", lib().dg_make_plan(int(mode), int(rows), int(N), int(K), int(G), int(num_sms),
                                               ctypes.byref(pl)))
     return pl.as_dict()
+
+
+def dg_selftest_bounded_wait(stream=None) -> None:
+    """Enqueue the bounded-wait self-test kernel (sets DG_DEVERR_TIMEOUT after ~1 s)."""
+    _check("dg_selftest_bounded_wait", lib().dg_selftest_bounded_wait(_stream(stream)))
 
 
 def dg_status_string(status: int) -> str:

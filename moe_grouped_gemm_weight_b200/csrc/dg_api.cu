@@ -13,6 +13,22 @@
 
 #include "dg.h"
 #include "dg_kernel.cuh"
+#include "dg_kernel_small.cuh"
+
+namespace dg {
+// One CTA waits (bounded) on a barrier that no one arrives at.
+__global__ void bounded_wait_selftest_kernel() {
+    __shared__ uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        abort_flag = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) mbar_wait(&bar, 0, &abort_flag);
+}
+}  // namespace dg
 
 namespace {
 
@@ -184,13 +200,56 @@ dg_status check_sizes(int mode, int rows, int N, int K, int G) {
     return DG_OK;
 }
 
-dg_status plan(int mode, int rows, int N, int K, int G, int num_sms, dg_plan* out) {
+// Few-row problems (dense M <= 128, masked M_max <= 256) go to the swap-AB
+// split-K kernel: TN activation rows per tile (the smallest of 32/64/128 that
+// holds them), 128 weight rows per tile, and as many K splits (cluster size,
+// at most 8 and at most K/128) as keep two CTAs on every SM busy.
+bool use_small(int mode, int rows) { return (mode == 0 && rows <= 128) || (mode == 2 && rows <= 256); }
+
+int small_tn(int mode, int rows) {
+    const int t = mode == 2 ? (rows < 128 ? rows : 128) : rows;
+    return t <= 32 ? 32 : t <= 64 ? 64 : 128;
+}
+
+int small_smem(int tn) {
+    return tn == 32 ? dg::small_smem_bytes<32>() : tn == 64 ? dg::small_smem_bytes<64>() : dg::small_smem_bytes<128>();
+}
+
+int small_stages(int tn) {
+    return tn == 32 ? dg::SmallCfg<32>::kStages : tn == 64 ? dg::SmallCfg<64>::kStages : dg::SmallCfg<128>::kStages;
+}
+
+dg_status plan(int mode, int rows, int N, int K, int G, int num_sms, dg_plan* out, int expected_m = 0) {
     dg_status s = check_sizes(mode, rows, N, K, G);
     if (s != DG_OK) return s;
     if (num_sms <= 0) return fail(DG_ERR_INVALID_ARG, "num_sms must be positive");
+    *out = dg_plan{};
+    if (use_small(mode, rows)) {
+        const int tn = small_tn(mode, rows);
+        const int per_group = cdiv(rows, tn);
+        const int m_blocks = mode == 2 ? G * per_group : per_group;
+        const int n_blocks = cdiv(N, 128);
+        // Masked: tiles past masked_m exit at once; with a hint, count only the
+        // tiles expected to hold rows.
+        int active_m = m_blocks;
+        if (mode == 2 && expected_m > 0) active_m = G * cdiv(expected_m < rows ? expected_m : rows, tn);
+        const long units = static_cast<long>(active_m) * n_blocks;
+        int split = static_cast<int>((2L * num_sms) / (units > 0 ? units : 1));
+        const int max_split = dg::kSmallMaxSplit < K / dg::kBK ? dg::kSmallMaxSplit : K / dg::kBK;
+        split = split < 1 ? 1 : (split > max_split ? max_split : split);
+        out->block_m = tn;
+        out->block_n = 128;
+        out->stages = small_stages(tn);
+        out->m_blocks = m_blocks;
+        out->n_blocks = n_blocks;
+        out->tiles = m_blocks * n_blocks;
+        out->grid = out->tiles * split;
+        out->smem_bytes = small_smem(tn);
+        out->swap_ab = 1;
+        out->split_k = split;
+        return DG_OK;
+    }
     const int m_blocks = (mode == 2) ? G * cdiv(rows, dg::kBM) : cdiv(rows, dg::kBM);
-    // Masked: the host does not know masked_m, so plan for every group being
-    // half full (or for expected_m, see dg_grouped_masked_nt).
     const Choice c = choose(m_blocks, N, num_sms);
     out->block_m = dg::kBM;
     out->block_n = c.bn;
@@ -200,6 +259,8 @@ dg_status plan(int mode, int rows, int N, int K, int G, int num_sms, dg_plan* ou
     out->tiles = m_blocks * out->n_blocks;
     out->grid = (mode == 2) ? num_sms : (out->tiles < num_sms ? out->tiles : num_sms);
     out->smem_bytes = plan_smem(c);
+    out->swap_ab = 0;
+    out->split_k = 1;
     return DG_OK;
 }
 
@@ -223,6 +284,50 @@ dg_status launch_one(const dg::Params& p, const CUtensorMap& ta, const CUtensorM
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return fail(DG_ERR_CUDA, "kernel launch failed: %s", cudaGetErrorString(e));
     return ok();
+}
+
+template <int TN, int MODE>
+dg_status launch_small(const dg::Params& p, const CUtensorMap& ta, const CUtensorMap& tb, const dg_plan& pl,
+                       cudaStream_t stream) {
+    constexpr int smem = dg::small_smem_bytes<TN>();
+    static_assert(smem <= 113 * 1024, "two CTAs per SM need <= 113 KiB each");
+    auto kern = dg::fp8_gemm_swapab_kernel<TN, MODE>;
+    static std::atomic<int> attr_set[kMaxDevices];
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev >= 0 && dev < kMaxDevices && !attr_set[dev].load()) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+            return fail(DG_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(cudaGetLastError()));
+        attr_set[dev].store(1);
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(pl.split_k), static_cast<unsigned>(pl.n_blocks),
+                       static_cast<unsigned>(pl.m_blocks));
+    cfg.blockDim = dim3(dg::kSmallThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = static_cast<unsigned>(pl.split_k);
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kern, p, ta, tb);
+    if (e == cudaSuccess) e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(DG_ERR_CUDA, "kernel launch failed: %s", cudaGetErrorString(e));
+    return ok();
+}
+
+template <int MODE>
+dg_status dispatch_small(const dg_plan& pl, const dg::Params& p, const CUtensorMap& ta, const CUtensorMap& tb,
+                         cudaStream_t stream) {
+    switch (pl.block_m) {
+        case 32: return launch_small<32, MODE>(p, ta, tb, pl, stream);
+        case 64: return launch_small<64, MODE>(p, ta, tb, pl, stream);
+        case 128: return launch_small<128, MODE>(p, ta, tb, pl, stream);
+        default: return fail(DG_ERR_UNSUPPORTED, "no few-row kernel for block_m=%d", pl.block_m);
+    }
 }
 
 template <int MODE>
@@ -253,6 +358,22 @@ dg_status common_checks(const void* D, const void* A, const float* sa, int sa_st
     return DG_OK;
 }
 
+// Raster group (m-blocks whose tiles run together, m fastest): B is streamed
+// from HBM once per group, so the group should be as tall as possible while
+// the group's A rows plus the weight tiles in flight across the grid
+// (grid / group of them) still fit in L2 (budget 96 MiB of the 126 MB).
+int choose_raster(int m_blocks, int n_blocks, int block_n, int K, int grid) {
+    const double budget = 96.0 * 1024 * 1024;
+    int best = 1;
+    for (int gm = 1; gm <= m_blocks; gm *= 2) {
+        const double a_bytes = static_cast<double>(gm) * dg::kBM * K;
+        const int active_n = n_blocks < cdiv(grid, gm) ? n_blocks : cdiv(grid, gm);
+        const double b_bytes = static_cast<double>(active_n) * block_n * K;
+        if (a_bytes + b_bytes <= budget) best = gm;
+    }
+    return best;
+}
+
 dg::Params make_params(uint16_t* D, const float* sa, int sa_stride, const float* sb, int rows, int N, int K, int G,
                        const dg_plan& pl) {
     dg::Params p{};
@@ -268,7 +389,7 @@ dg::Params make_params(uint16_t* D, const float* sa, int sa_stride, const float*
     p.nbn = cdiv(N, 128);
     p.n_blocks = pl.n_blocks;
     p.m_blocks = pl.m_blocks;
-    p.raster = 8;
+    p.raster = pl.swap_ab ? 1 : choose_raster(pl.m_blocks, pl.n_blocks, pl.block_n, K, pl.grid);
     p.b_stream = 0;
     return p;
 }
@@ -288,6 +409,12 @@ dg_status dg_fp8_gemm_nt(uint16_t* D, const uint8_t* A, const float* sa, int sa_
     dg_plan pl;
     if ((s = plan(0, M, N, K, 1, sms, &pl)) != DG_OK) return s;
     CUtensorMap ta, tb;
+    if (pl.swap_ab) {
+        if ((s = make_operand_map(&ta, A, K, M, 1, pl.block_m, false)) != DG_OK) return s;
+        if ((s = make_operand_map(&tb, B, K, N, 1, 128, true)) != DG_OK) return s;
+        dg::Params p = make_params(D, sa, sa_stride, sb, M, N, K, 1, pl);
+        return dispatch_small<dg::kDense>(pl, p, ta, tb, static_cast<cudaStream_t>(stream));
+    }
     if ((s = make_operand_map(&ta, A, K, M, 1, dg::kBM, false)) != DG_OK) return s;
     if ((s = make_operand_map(&tb, B, K, N, 1, pl.block_n, true)) != DG_OK) return s;
     CUtensorMap td;
@@ -322,7 +449,6 @@ dg_status dg_grouped_contiguous_nt(uint16_t* D, const uint8_t* A, const float* s
 dg_status dg_grouped_masked_nt(uint16_t* D, const uint8_t* A, const float* sa, int sa_stride, const uint8_t* B,
                                const float* sb, const int32_t* masked_m, int G, int M_max, int N, int K,
                                int expected_m, void* stream) {
-    (void)expected_m;
     dg_status s = check_sizes(2, M_max, N, K, G);
     if (s != DG_OK) return s;
     if ((s = common_checks(D, A, sa, sa_stride, B, sb, M_max)) != DG_OK) return s;
@@ -331,8 +457,16 @@ dg_status dg_grouped_masked_nt(uint16_t* D, const uint8_t* A, const float* sa, i
     const int sms = effective_sms();
     if (sms <= 0) return fail(DG_ERR_CUDA, "no CUDA device");
     dg_plan pl;
-    if ((s = plan(2, M_max, N, K, G, sms, &pl)) != DG_OK) return s;
+    if ((s = plan(2, M_max, N, K, G, sms, &pl, expected_m)) != DG_OK) return s;
     CUtensorMap ta, tb;
+    if (pl.swap_ab) {
+        if ((s = make_operand_map(&ta, A, K, M_max, G, pl.block_m, true)) != DG_OK) return s;
+        if ((s = make_operand_map(&tb, B, K, N, G, 128, true)) != DG_OK) return s;
+        dg::Params p = make_params(D, sa, sa_stride, sb, M_max, N, K, G, pl);
+        p.masked_m = masked_m;
+        p.m_blocks = pl.m_blocks / G;  // TN-row blocks per group
+        return dispatch_small<dg::kMasked>(pl, p, ta, tb, static_cast<cudaStream_t>(stream));
+    }
     if ((s = make_operand_map(&ta, A, K, M_max, G, dg::kBM, true)) != DG_OK) return s;
     if ((s = make_operand_map(&tb, B, K, N, G, pl.block_n, true)) != DG_OK) return s;
     CUtensorMap td;
@@ -364,6 +498,13 @@ dg_status dg_get_device_error(int* code) {
     if (e == cudaSuccess) e = cudaMemcpyToSymbol(dg::g_dg_error, &zero, sizeof(zero));
     if (e != cudaSuccess) return fail(DG_ERR_CUDA, "reading the device error word: %s", cudaGetErrorString(e));
     *code = static_cast<int>(v);
+    return ok();
+}
+
+dg_status dg_selftest_bounded_wait(void* stream) {
+    dg::bounded_wait_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>();
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(DG_ERR_CUDA, "self-test launch failed: %s", cudaGetErrorString(e));
     return ok();
 }
 

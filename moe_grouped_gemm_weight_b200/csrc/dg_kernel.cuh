@@ -302,39 +302,40 @@ fp8_gemm_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtens
         __syncwarp();
     } else if (warp == 2) {
         // ------------------------------------------------ scale producer ----
+        // Per K block: lane l copies sa rows m0+4l..m0+4l+3 (16 bytes) and
+        // lanes 0..3 the tile's sb values; the copies run asynchronously and
+        // complete the slot's barrier when they land, so this warp only ever
+        // waits for a free slot.  Rows past the data and sb blocks past N are
+        // zero-filled, nothing outside the tensors is read.
         int slot = 0;
         uint32_t sphase = 0;
-        bool ok = true;
         const int row_limit = p.M;  // rows of sa that exist (dense M, M_total or M_max)
-        for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
+        for (int t = blockIdx.x; t < tiles; t += gridDim.x) {
             const Tile tl = decode_tile<BN, MODE>(p, t, m_blocks, mb_prefix);
             if (!tl.valid) continue;
             const float* sa_base = p.sa + (MODE == kMasked ? static_cast<int64_t>(tl.g) * nkb * p.sa_stride : 0);
             const float* sb_g = p.sb + static_cast<int64_t>(tl.g) * p.nbn * nkb;
-            const int nb_first = tl.n0 / 128;
+            const int nb = tl.n0 / 128 + (lane & 3);
+            const bool nb_ok = nb < p.nbn;
             const int r4 = tl.m0 + lane * 4;
+            const int left = row_limit - r4;
+            const uint32_t sa_bytes = left >= 4 ? 16u : (left > 0 ? static_cast<uint32_t>(left) * 4u : 0u);
+            bool ok = true;
             for (int kb = 0; kb < nkb; ++kb) {
                 if (!mbar_wait(sempty + slot, sphase ^ 1u, abort_flag)) { ok = false; break; }
-                const float* src = sa_base + static_cast<int64_t>(kb) * p.sa_stride + r4;
-                float4 v;
-                if (r4 + 3 < row_limit) {
-                    v = ld_nc_f4(src);
-                } else {
-                    v.x = r4 + 0 < row_limit ? __ldg(src + 0) : 0.f;
-                    v.y = r4 + 1 < row_limit ? __ldg(src + 1) : 0.f;
-                    v.z = r4 + 2 < row_limit ? __ldg(src + 2) : 0.f;
-                    v.w = r4 + 3 < row_limit ? __ldg(src + 3) : 0.f;
-                }
-                float* dst = sring + slot * kScaleSlotFloats;
-                *reinterpret_cast<float4*>(dst + lane * 4) = v;
-                if (lane < 4) {
-                    const int nb = min(nb_first + lane, p.nbn - 1);
-                    dst[kBM + lane] = __ldg(sb_g + static_cast<int64_t>(nb) * nkb + kb);
-                }
-                mbar_arrive(sfull + slot);
+                const uint32_t dst = smem_u32(sring + slot * kScaleSlotFloats);
+                const float* src = sa_bytes ? sa_base + static_cast<int64_t>(kb) * p.sa_stride + r4 : p.sa;
+                cp_async_16(dst + lane * 16, src, sa_bytes);
+                if (lane < 4)
+                    cp_async_4(dst + (kBM + lane) * 4, nb_ok ? sb_g + static_cast<int64_t>(nb) * nkb + kb : p.sb,
+                               nb_ok ? 4u : 0u);
+                cp_async_arrive(sfull + slot);
                 if (++slot == kScaleSlots) { slot = 0; sphase ^= 1u; }
             }
+            if (!ok) break;
         }
+        // Let every copy land before the CTA can exit.
+        asm volatile("cp.async.wait_all;" ::: "memory");
     }
     } else {
         // ------------------------------------------ promotion + epilogue ----

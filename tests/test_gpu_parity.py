@@ -259,3 +259,31 @@ def test_masked_under_cuda_graph_follows_device_counts(dgm):
         for gi, m in enumerate(counts):
             assert_close(got[gi, :m], ref[gi, :m], mag[gi, :m], f"graph replay g={gi}")
     assert dgm.dg_get_device_error() == 0
+
+
+# ------------------------------------------------- few-row (swap-AB) kernel --
+
+@pytest.mark.parametrize("M", [1, 17, 32, 33, 64, 100, 128])
+@pytest.mark.parametrize("sms", [148, 16, 3])
+def test_few_rows_split_k_variants(dgm, M, sms):
+    N, K = 520, 1536
+    c = wl.dense_case(M, N, K, seed=M * 3 + sms)
+    try:
+        dgm.dg_set_num_sms(sms)
+        plan = dgm.dg_make_plan(0, M, N, K, 1, sms)
+        assert plan["swap_ab"] == 1
+        got = run_dense(dgm, c)
+    finally:
+        dgm.dg_set_num_sms(0)
+    ref, mag = oracle_dense(c)
+    assert_close(got, ref, mag, f"few rows M={M} split={plan['split_k']}")
+
+
+def test_few_rows_k_split_uneven(dgm):
+    # 7 K blocks over a cluster of up to 8 CTAs: some CTAs own one block, the
+    # split sizes differ, and the fixed-order sum must still match.
+    c = wl.dense_case(64, 2112, 896, seed=21)
+    got = run_dense(dgm, c)
+    ref, mag = oracle_dense(c)
+    assert_close(got, ref, mag, "uneven split")
+    assert dgm.dg_make_plan(0, 64, 2112, 896, 1, 148)["split_k"] == 7

@@ -76,17 +76,37 @@ def test_plan_reproduces_the_pages_block_count_arithmetic():
 
 
 @pytest.mark.parametrize("mode,rows,N,K,G", [(0, 64, 2112, 7168, 1), (0, 4096, 7168, 16384, 1),
-                                            (1, 32768, 4096, 7168, 4), (2, 256, 4096, 7168, 4)])
+                                            (1, 32768, 4096, 7168, 4), (2, 256, 4096, 7168, 4),
+                                            (2, 1024, 4096, 7168, 1), (0, 129, 512, 1024, 1)])
 def test_plan_is_consistent(mode, rows, N, K, G):
     p = dg.dg_make_plan(mode, rows, N, K, G, 148)
-    assert p["block_n"] in (64, 128, 192, 256)
     assert p["n_blocks"] == -(-N // p["block_n"])
-    mb = -(-rows // 128) * (G if mode == 2 else 1)
+    mb = -(-rows // p["block_m"]) * (G if mode == 2 else 1)
     assert p["m_blocks"] == mb
     assert p["tiles"] == mb * p["n_blocks"]
-    assert 1 <= p["grid"] <= 148
-    assert p["smem_bytes"] <= 227 * 1024
     assert p["stages"] >= 2
+    if p["swap_ab"]:
+        # Few-row kernel: 128 weight rows per tile, one cluster of split_k CTAs
+        # per tile, two CTAs per SM.
+        assert rows <= (256 if mode == 2 else 128)
+        assert p["block_n"] == 128 and p["block_m"] in (32, 64, 128)
+        assert 1 <= p["split_k"] <= min(8, K // 128)
+        assert p["grid"] == p["tiles"] * p["split_k"]
+        assert p["smem_bytes"] <= 113 * 1024
+    else:
+        assert p["block_m"] == 128 and p["block_n"] in (64, 128, 256)
+        assert p["split_k"] == 1
+        assert 1 <= p["grid"] <= 148
+        assert p["smem_bytes"] <= 227 * 1024
+
+
+@pytest.mark.parametrize("M,tn", [(1, 32), (32, 32), (33, 64), (64, 64), (65, 128), (128, 128)])
+def test_few_row_plan_tile_and_split(M, tn):
+    p = dg.dg_make_plan(0, M, 2112, 7168, 1, 148)
+    assert p["swap_ab"] == 1 and p["block_m"] == tn
+    # 17 weight tiles; as many K splits as keep two CTAs per SM busy, at most 8.
+    assert p["n_blocks"] == 17 and p["split_k"] == min(8, (2 * 148) // 17)
+    assert dg.dg_make_plan(0, 129, 2112, 7168, 1, 148)["swap_ab"] == 0
 
 
 @pytest.mark.parametrize("args,expect", [
