@@ -158,6 +158,7 @@ typedef struct dg_plan {
     int smem_bytes;   /* dynamic shared memory per CTA                           */
     int swap_ab;      /* 1: few-row kernel (weights on the MMA's 128-row side)   */
     int split_k;      /* CTAs (one thread-block cluster) sharing each tile's K   */
+    int cta_pair;     /* 1: 256x256 tiles on CTA pairs (tcgen05 cta_group::2)    */
 } dg_plan;
 
 DG_API dg_status dg_make_plan(int mode, int rows, int N, int K, int G, int num_sms, dg_plan* out);

@@ -7,6 +7,7 @@
 
 #include <atomic>
 #include <cstdarg>
+#include <cstdlib>
 #include <cstdio>
 #include <cstring>
 #include <mutex>
@@ -14,6 +15,7 @@
 #include "dg.h"
 #include "dg_kernel.cuh"
 #include "dg_kernel_small.cuh"
+#include "dg_kernel_pair.cuh"
 
 namespace dg {
 // One CTA waits (bounded) on a barrier that no one arrives at.
@@ -137,7 +139,13 @@ dg_status make_output_map(CUtensorMap* tm, void* base, int N, int rows, int grou
 struct Choice {
     int bn;
     int stages;
+    bool pair;
 };
+
+constexpr int kPairBN = 256;  // pair tile 256 x 256 (256 x 128 measured slower)
+constexpr int kPairStages = (227 * 1024 - 32 * 1024) / dg::PairCfg<kPairBN>::kStageBytes > 8
+                                ? 8
+                                : (227 * 1024 - 32 * 1024) / dg::PairCfg<kPairBN>::kStageBytes;
 
 // Ring depth: as many stages as fit in 227 KiB of shared memory, at most 8.
 template <int BN>
@@ -163,9 +171,9 @@ constexpr int smem_for() {
 // the DeepGEMM README page (section "非对齐的块大小"); here BN stays a
 // multiple of 64 so that the two promotion warpgroups split it into 32-column
 // TMEM loads.
-Choice choose(int m_blocks, int N, int num_sms) {
+Choice choose(int m_blocks, int pair_m_blocks, int N, int num_sms, bool pair_ok) {
     const int cands[3] = {256, 128, 64};
-    Choice best{128, max_stages<128>()};
+    Choice best{128, max_stages<128>(), false};
     double best_cost = -1.0;
     for (int bn : cands) {
         const int tiles = m_blocks * cdiv(N, bn);
@@ -176,11 +184,25 @@ Choice choose(int m_blocks, int N, int num_sms) {
             best.bn = bn;
         }
     }
-    best.stages = best.bn == 256 ? max_stages<256>() : best.bn == 128 ? max_stages<128>() : max_stages<64>();
+    // CTA pairs: a 256 x 256 tile on two SMs; per SM and K block the MMA work
+    // of a 128 x 256 tile with 32 KiB (128 + 128 rows) of operands.
+    if (pair_ok && num_sms >= 2) {
+        const int pair_tiles = pair_m_blocks * cdiv(N, kPairBN);
+        // per SM and K block: 128 x kPairBN MMA work, 128 + kPairBN/2 operand rows
+        const double mma = kPairBN, load = 0.75 * (128 + kPairBN / 2);
+        const double t_kb = mma > load ? mma : load;
+        const double cost = static_cast<double>(waves_cost(pair_tiles, num_sms / 2)) * t_kb;
+        best_cost = cost;
+        best.bn = kPairBN;
+        best.pair = true;
+    }
+    best.stages = best.pair ? kPairStages
+                            : best.bn == 256 ? max_stages<256>() : best.bn == 128 ? max_stages<128>() : max_stages<64>();
     return best;
 }
 
 int plan_smem(const Choice& c) {
+    if (c.pair) return dg::pair_smem_bytes<kPairBN, kPairStages>();
     return c.bn == 256 ? smem_for<256>() : c.bn == 128 ? smem_for<128>() : smem_for<64>();
 }
 
@@ -250,7 +272,31 @@ dg_status plan(int mode, int rows, int N, int K, int G, int num_sms, dg_plan* ou
         return DG_OK;
     }
     const int m_blocks = (mode == 2) ? G * cdiv(rows, dg::kBM) : cdiv(rows, dg::kBM);
-    const Choice c = choose(m_blocks, N, num_sms);
+    // Pairs need every 256-row tile inside one group: dense, or masked (groups
+    // are separate blocks of M_max rows); not the contiguous layout, whose
+    // segments are only 128-row aligned.
+    // CTA pairs are measured no faster than single-CTA 128 x 256 tiles on the
+    // dense sweep, so they are used only when DG_FORCE_PAIR=1 (experiments).
+    const char* force_pair = std::getenv("DG_FORCE_PAIR");
+    const bool pairs = force_pair && force_pair[0] == '1' && mode != 1;
+    const int pair_m_blocks = (mode == 2 ? G : 1) * cdiv(rows, dg::kPairBM);
+    const Choice c = choose(m_blocks, pair_m_blocks, N, num_sms, pairs);
+    if (c.pair) {
+        const int per_group = cdiv(rows, dg::kPairBM);
+        out->block_m = dg::kPairBM;
+        out->block_n = kPairBN;
+        out->stages = c.stages;
+        out->m_blocks = mode == 2 ? G * per_group : per_group;
+        out->n_blocks = cdiv(N, kPairBN);
+        out->tiles = out->m_blocks * out->n_blocks;
+        const int pairs = num_sms / 2;
+        out->grid = 2 * ((mode == 2 || out->tiles > pairs) ? pairs : out->tiles);
+        out->smem_bytes = plan_smem(c);
+        out->swap_ab = 0;
+        out->split_k = 1;
+        out->cta_pair = 1;
+        return DG_OK;
+    }
     out->block_m = dg::kBM;
     out->block_n = c.bn;
     out->stages = c.stages;
@@ -261,6 +307,7 @@ dg_status plan(int mode, int rows, int N, int K, int G, int num_sms, dg_plan* ou
     out->smem_bytes = plan_smem(c);
     out->swap_ab = 0;
     out->split_k = 1;
+    out->cta_pair = 0;
     return DG_OK;
 }
 
@@ -282,6 +329,77 @@ dg_status launch_one(const dg::Params& p, const CUtensorMap& ta, const CUtensorM
     }
     kern<<<grid, dg::kThreads, smem, stream>>>(p, ta, tb, td);
     cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(DG_ERR_CUDA, "kernel launch failed: %s", cudaGetErrorString(e));
+    return ok();
+}
+
+// How many 2-CTA clusters of the pair kernel can be resident at once (a
+// cluster must fit inside one GPC, so this can be below SMs / 2).  Cached per
+// device; 0 if the query fails.
+template <int MODE>
+int pair_max_active_clusters() {
+    static std::atomic<int> cached[kMaxDevices];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 0;
+    int n = cached[dev].load();
+    if (n > 0) return n;
+    constexpr int smem = dg::pair_smem_bytes<kPairBN, kPairStages>();
+    auto kern = dg::fp8_gemm_pair_kernel<kPairBN, kPairStages, MODE>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) {
+        cudaGetLastError();
+        return 0;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * 74, 1, 1);
+    cfg.blockDim = dim3(dg::kThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) {
+        cudaGetLastError();
+        return 0;
+    }
+    cached[dev].store(n);
+    return n;
+}
+
+template <int MODE>
+dg_status launch_pair(const dg::Params& p, const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& td,
+                      const dg_plan& pl, cudaStream_t stream) {
+    constexpr int smem = dg::pair_smem_bytes<kPairBN, kPairStages>();
+    static_assert(smem <= 227 * 1024, "shared memory budget exceeded");
+    auto kern = dg::fp8_gemm_pair_kernel<kPairBN, kPairStages, MODE>;
+    static std::atomic<int> attr_set[kMaxDevices];
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev >= 0 && dev < kMaxDevices && !attr_set[dev].load()) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+            return fail(DG_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(cudaGetLastError()));
+        attr_set[dev].store(1);
+    }
+    // Persistent grid: never more clusters than can be resident together.
+    int grid = pl.grid;
+    const int max_clusters = pair_max_active_clusters<MODE>();
+    if (max_clusters > 0 && grid > 2 * max_clusters) grid = 2 * max_clusters;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
+    cfg.blockDim = dim3(dg::kThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kern, p, ta, tb, td);
+    if (e == cudaSuccess) e = cudaGetLastError();
     if (e != cudaSuccess) return fail(DG_ERR_CUDA, "kernel launch failed: %s", cudaGetErrorString(e));
     return ok();
 }
@@ -362,11 +480,11 @@ dg_status common_checks(const void* D, const void* A, const float* sa, int sa_st
 // from HBM once per group, so the group should be as tall as possible while
 // the group's A rows plus the weight tiles in flight across the grid
 // (grid / group of them) still fit in L2 (budget 96 MiB of the 126 MB).
-int choose_raster(int m_blocks, int n_blocks, int block_n, int K, int grid) {
+int choose_raster(int m_blocks, int n_blocks, int block_m, int block_n, int K, int grid) {
     const double budget = 96.0 * 1024 * 1024;
     int best = 1;
     for (int gm = 1; gm <= m_blocks; gm *= 2) {
-        const double a_bytes = static_cast<double>(gm) * dg::kBM * K;
+        const double a_bytes = static_cast<double>(gm) * block_m * K;
         const int active_n = n_blocks < cdiv(grid, gm) ? n_blocks : cdiv(grid, gm);
         const double b_bytes = static_cast<double>(active_n) * block_n * K;
         if (a_bytes + b_bytes <= budget) best = gm;
@@ -389,7 +507,9 @@ dg::Params make_params(uint16_t* D, const float* sa, int sa_stride, const float*
     p.nbn = cdiv(N, 128);
     p.n_blocks = pl.n_blocks;
     p.m_blocks = pl.m_blocks;
-    p.raster = pl.swap_ab ? 1 : choose_raster(pl.m_blocks, pl.n_blocks, pl.block_n, K, pl.grid);
+    p.raster = pl.swap_ab ? 1
+                          : choose_raster(pl.m_blocks, pl.n_blocks, pl.block_m, pl.block_n, K,
+                                          pl.cta_pair ? pl.grid / 2 : pl.grid);
     p.b_stream = 0;
     return p;
 }
@@ -416,11 +536,12 @@ dg_status dg_fp8_gemm_nt(uint16_t* D, const uint8_t* A, const float* sa, int sa_
         return dispatch_small<dg::kDense>(pl, p, ta, tb, static_cast<cudaStream_t>(stream));
     }
     if ((s = make_operand_map(&ta, A, K, M, 1, dg::kBM, false)) != DG_OK) return s;
-    if ((s = make_operand_map(&tb, B, K, N, 1, pl.block_n, true)) != DG_OK) return s;
+    if ((s = make_operand_map(&tb, B, K, N, 1, pl.cta_pair ? pl.block_n / 2 : pl.block_n, true)) != DG_OK) return s;
     CUtensorMap td;
     if ((s = make_output_map(&td, D, N, M, 1, false)) != DG_OK) return s;
     dg::Params p = make_params(D, sa, sa_stride, sb, M, N, K, 1, pl);
     p.b_stream = pl.m_blocks == 1;
+    if (pl.cta_pair) return launch_pair<dg::kDense>(p, ta, tb, td, pl, static_cast<cudaStream_t>(stream));
     return dispatch<dg::kDense>(pl, p, ta, tb, td, static_cast<cudaStream_t>(stream));
 }
 
@@ -468,12 +589,13 @@ dg_status dg_grouped_masked_nt(uint16_t* D, const uint8_t* A, const float* sa, i
         return dispatch_small<dg::kMasked>(pl, p, ta, tb, static_cast<cudaStream_t>(stream));
     }
     if ((s = make_operand_map(&ta, A, K, M_max, G, dg::kBM, true)) != DG_OK) return s;
-    if ((s = make_operand_map(&tb, B, K, N, G, pl.block_n, true)) != DG_OK) return s;
+    if ((s = make_operand_map(&tb, B, K, N, G, pl.cta_pair ? pl.block_n / 2 : pl.block_n, true)) != DG_OK) return s;
     CUtensorMap td;
     if ((s = make_output_map(&td, D, N, M_max, G, true)) != DG_OK) return s;
     dg::Params p = make_params(D, sa, sa_stride, sb, M_max, N, K, G, pl);
     p.masked_m = masked_m;
     p.b_stream = M_max <= dg::kBM;
+    if (pl.cta_pair) return launch_pair<dg::kMasked>(p, ta, tb, td, pl, static_cast<cudaStream_t>(stream));
     return dispatch<dg::kMasked>(pl, p, ta, tb, td, static_cast<cudaStream_t>(stream));
 }
 

@@ -287,3 +287,40 @@ def test_few_rows_k_split_uneven(dgm):
     ref, mag = oracle_dense(c)
     assert_close(got, ref, mag, "uneven split")
     assert dgm.dg_make_plan(0, 64, 2112, 896, 1, 148)["split_k"] == 7
+
+
+# ------------------------------------------- CTA-pair kernel (opt-in path) --
+
+@pytest.fixture
+def force_pair(monkeypatch):
+    monkeypatch.setenv("DG_FORCE_PAIR", "1")
+    yield
+
+
+@pytest.mark.parametrize("M,N,K", [(256, 256, 128), (300, 520, 640), (513, 264, 1024), (129, 136, 256)])
+def test_pair_kernel_dense_full(dgm, force_pair, M, N, K):
+    assert dgm.dg_make_plan(0, M, N, K, 1, 148)["cta_pair"] == 1
+    c = wl.dense_case(M, N, K, seed=M + N + K + 1)
+    got = run_dense(dgm, c)
+    ref, mag = oracle_dense(c)
+    assert_close(got, ref, mag, f"pair dense {M}x{N}x{K}")
+
+
+def test_pair_kernel_dense_large_sampled(dgm, force_pair):
+    c = wl.dense_case(4096, 7168, 2048, seed=0, device="cuda").to("cpu")
+    got = run_dense(dgm, c)
+    rows = sample_rows(4096, seed=8, extra=(255, 256, 383, 384))
+    ref, mag = oracle_dense(c, rows=rows)
+    assert_close(got[rows], ref[rows], mag[rows], "pair dense 4096x7168x2048")
+
+
+def test_pair_kernel_masked_full(dgm, force_pair):
+    mm = [300, 0, 257, 1]
+    c = wl.masked_case(4, 300, 264, 512, masked_m=mm, seed=31)
+    assert dgm.dg_make_plan(2, 300, 264, 512, 4, 148)["cta_pair"] == 1
+    got = run_masked(dgm, c)
+    check_masked_untouched(got, mm)
+    ref, mag = oracle_masked(c)
+    for g in range(4):
+        assert_close(got[g, :mm[g]], ref[g, :mm[g]], mag[g, :mm[g]], f"pair masked g={g}")
+    assert dgm.dg_get_device_error() == 0
