@@ -18,6 +18,14 @@
  *  Pointers   All tensor pointers are CUDA DEVICE pointers, 16-byte aligned,
  *             owned by the caller.  The library never allocates, frees or
  *             keeps them past the call.
+ *  Workspace  Dense calls whose last wave of tiles is partial split those
+ *             tiles along K; the slices' FP32 partials go to a workspace the
+ *             library allocates ONCE per (device, stream) on first need (one
+ *             128 x BN FP32 tile per SM, about 19 MB on a B200, zeroed) and
+ *             keeps until exit.  While a stream is being captured into a CUDA
+ *             graph and has no workspace yet, calls do not split (results are
+ *             the same up to FP32 summation order); make one call on the
+ *             stream before capturing to keep the split.
  *  Layouts    A   uint8 (e4m3 codes) [rows][K], K contiguous.
  *             B   uint8 (e4m3 codes) [G][N][K], K contiguous ("NT": the RHS is
  *                 stored transposed).  G = 1 for the dense call.
@@ -159,6 +167,8 @@ typedef struct dg_plan {
     int swap_ab;      /* 1: few-row kernel (weights on the MMA's 128-row side)   */
     int split_k;      /* CTAs (one thread-block cluster) sharing each tile's K   */
     int cta_pair;     /* 1: 256x256 tiles on CTA pairs (tcgen05 cta_group::2)    */
+    int tail_split;   /* >1: the tiles of the last partial wave are split into   */
+                      /* this many K slices (dense calls only; 1 = off)          */
 } dg_plan;
 
 DG_API dg_status dg_make_plan(int mode, int rows, int N, int K, int G, int num_sms, dg_plan* out);

@@ -8,6 +8,9 @@
 #include <atomic>
 #include <cstdarg>
 #include <cstdlib>
+#include <cmath>
+#include <map>
+#include <utility>
 #include <cstdio>
 #include <cstring>
 #include <mutex>
@@ -172,6 +175,8 @@ constexpr int smem_for() {
 // multiple of 64 so that the two promotion warpgroups split it into 32-column
 // TMEM loads.
 Choice choose(int m_blocks, int pair_m_blocks, int N, int num_sms, bool pair_ok) {
+    // 192 (three promotion warpgroups) is measured ~12% slower per tile than
+    // 256 on the dense sweep: reachable with DG_FORCE_BN, not chosen.
     const int cands[3] = {256, 128, 64};
     Choice best{128, max_stages<128>(), false};
     double best_cost = -1.0;
@@ -196,14 +201,23 @@ Choice choose(int m_blocks, int pair_m_blocks, int N, int num_sms, bool pair_ok)
         best.bn = kPairBN;
         best.pair = true;
     }
+    // DG_FORCE_BN=64|128|192|256 pins the single-CTA tile width (experiments).
+    const char* force_bn = std::getenv("DG_FORCE_BN");
+    if (force_bn && !best.pair) {
+        const int f = std::atoi(force_bn);
+        if (f == 64 || f == 128 || f == 192 || f == 256) best.bn = f;
+    }
     best.stages = best.pair ? kPairStages
-                            : best.bn == 256 ? max_stages<256>() : best.bn == 128 ? max_stages<128>() : max_stages<64>();
+                            : best.bn == 256 ? max_stages<256>()
+                            : best.bn == 192 ? max_stages<192>()
+                            : best.bn == 128 ? max_stages<128>()
+                                             : max_stages<64>();
     return best;
 }
 
 int plan_smem(const Choice& c) {
     if (c.pair) return dg::pair_smem_bytes<kPairBN, kPairStages>();
-    return c.bn == 256 ? smem_for<256>() : c.bn == 128 ? smem_for<128>() : smem_for<64>();
+    return c.bn == 256 ? smem_for<256>() : c.bn == 192 ? smem_for<192>() : c.bn == 128 ? smem_for<128>() : smem_for<64>();
 }
 
 dg_status check_sizes(int mode, int rows, int N, int K, int G) {
@@ -308,6 +322,26 @@ dg_status plan(int mode, int rows, int N, int K, int G, int num_sms, dg_plan* ou
     out->swap_ab = 0;
     out->split_k = 1;
     out->cta_pair = 0;
+    out->tail_split = 1;
+    // Dense: when the last wave is partial (R leftover tiles after W full
+    // waves), split each leftover tile into S K slices run by the idle CTAs.
+    // A slice takes ~nkb/S K blocks; slice 0 then reads S-1 partial tiles
+    // (each costs about 1.5 K blocks' time), so S ~ sqrt(nkb / 1.5) balances
+    // the two; also S*R <= grid, S <= 8 and at least 16 K blocks per slice.
+    if (mode == 0) {
+        const int waves = out->tiles / out->grid;
+        const int rest = out->tiles - waves * out->grid;
+        const int nkb = K / dg::kBK;
+        if (waves >= 1 && rest > 0) {
+            int split = static_cast<int>(std::sqrt(nkb / 1.5) + 0.5);
+            if (split > out->grid / rest) split = out->grid / rest;
+            if (split > 8) split = 8;
+            // Slices shorter than 16 K blocks do not repay the partial
+            // write, the flag hand-off and the reduction (measured).
+            if (split > nkb / 16) split = nkb / 16;
+            if (split >= 2) out->tail_split = split;
+        }
+    }
     return DG_OK;
 }
 
@@ -327,7 +361,7 @@ dg_status launch_one(const dg::Params& p, const CUtensorMap& ta, const CUtensorM
             return fail(DG_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(cudaGetLastError()));
         attr_set[dev].store(1);
     }
-    kern<<<grid, dg::kThreads, smem, stream>>>(p, ta, tb, td);
+    kern<<<grid, dg::Cfg<BN>::kThreadsC, smem, stream>>>(p, ta, tb, td);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return fail(DG_ERR_CUDA, "kernel launch failed: %s", cudaGetErrorString(e));
     return ok();
@@ -453,6 +487,7 @@ dg_status dispatch(const dg_plan& pl, const dg::Params& p, const CUtensorMap& ta
                    const CUtensorMap& td, cudaStream_t stream) {
     switch (pl.block_n) {
         case 256: return launch_one<256, max_stages<256>(), MODE>(p, ta, tb, td, pl.grid, stream);
+        case 192: return launch_one<192, max_stages<192>(), MODE>(p, ta, tb, td, pl.grid, stream);
         case 128: return launch_one<128, max_stages<128>(), MODE>(p, ta, tb, td, pl.grid, stream);
         case 64: return launch_one<64, max_stages<64>(), MODE>(p, ta, tb, td, pl.grid, stream);
         default: return fail(DG_ERR_UNSUPPORTED, "no kernel for block_n=%d", pl.block_n);
@@ -492,6 +527,54 @@ int choose_raster(int m_blocks, int n_blocks, int block_m, int block_n, int K, i
     return best;
 }
 
+// Workspace for the K-split tail: per (device, stream), allocated once on
+// first need, never during stream capture.  Holds one 128 x 256 FP32 partial
+// per SM (the split keeps fewer than grid <= SMs partials) and their flags.
+struct TailWorkspace {
+    float* partials = nullptr;
+    unsigned int* flags = nullptr;
+};
+
+bool tail_workspace(cudaStream_t stream, TailWorkspace* out) {
+    static std::mutex mu;
+    static std::map<std::pair<int, cudaStream_t>, TailWorkspace> spaces;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        return false;
+    }
+    std::lock_guard<std::mutex> lock(mu);
+    auto key = std::make_pair(dev, stream);
+    auto it = spaces.find(key);
+    if (it != spaces.end()) {
+        *out = it->second;
+        return true;
+    }
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(stream, &cs) != cudaSuccess) {
+        cudaGetLastError();
+        return false;
+    }
+    if (cs != cudaStreamCaptureStatusNone) return false;
+    const int sms = device_sm_count();
+    if (sms <= 0) return false;
+    TailWorkspace ws;
+    const size_t part_bytes = static_cast<size_t>(sms) * dg::kBM * 256 * sizeof(float);
+    const size_t flag_bytes = static_cast<size_t>(sms) * sizeof(unsigned int);
+    if (cudaMalloc(&ws.partials, part_bytes) != cudaSuccess) {
+        cudaGetLastError();
+        return false;
+    }
+    if (cudaMalloc(&ws.flags, flag_bytes) != cudaSuccess || cudaMemset(ws.flags, 0, flag_bytes) != cudaSuccess) {
+        cudaGetLastError();
+        cudaFree(ws.partials);
+        return false;
+    }
+    spaces[key] = ws;
+    *out = ws;
+    return true;
+}
+
 dg::Params make_params(uint16_t* D, const float* sa, int sa_stride, const float* sb, int rows, int N, int K, int G,
                        const dg_plan& pl) {
     dg::Params p{};
@@ -511,6 +594,8 @@ dg::Params make_params(uint16_t* D, const float* sa, int sa_stride, const float*
                           : choose_raster(pl.m_blocks, pl.n_blocks, pl.block_m, pl.block_n, K,
                                           pl.cta_pair ? pl.grid / 2 : pl.grid);
     p.b_stream = 0;
+    p.tail_split = 1;
+    p.full_tiles = pl.tiles;
     return p;
 }
 
@@ -542,6 +627,13 @@ dg_status dg_fp8_gemm_nt(uint16_t* D, const uint8_t* A, const float* sa, int sa_
     dg::Params p = make_params(D, sa, sa_stride, sb, M, N, K, 1, pl);
     p.b_stream = pl.m_blocks == 1;
     if (pl.cta_pair) return launch_pair<dg::kDense>(p, ta, tb, td, pl, static_cast<cudaStream_t>(stream));
+    TailWorkspace ws;
+    if (pl.tail_split > 1 && tail_workspace(static_cast<cudaStream_t>(stream), &ws)) {
+        p.tail_split = pl.tail_split;
+        p.full_tiles = (pl.tiles / pl.grid) * pl.grid;
+        p.ws = ws.partials;
+        p.ws_flags = ws.flags;
+    }
     return dispatch<dg::kDense>(pl, p, ta, tb, td, static_cast<cudaStream_t>(stream));
 }
 

@@ -61,18 +61,66 @@ struct Params {
     int m_blocks;   // dense/contiguous: ceil(M / 128); masked: unused (device prefix)
     int raster;     // m-blocks per raster group
     int b_stream;   // 1: B is read once (evict-first in L2), 0: B is reused
+    // K-split of the last partial wave (dense only; tail_split = 1: off).
+    // Tiles [0, full_tiles) go round-robin, whole K; each of the remaining
+    // tiles is split into tail_split K slices run by otherwise idle CTAs.
+    int full_tiles;
+    int tail_split;
+    float* ws;            // FP32 partials of slices 1..tail_split-1
+    unsigned int* ws_flags;  // one ready flag per partial
 };
 
+// One unit of work of this CTA: a tile (index t) over K blocks [kb0, kb1);
+// slice = -1 for a whole tile, else the K slice of a split tail tile.
+struct Work {
+    int t, kb0, kb1, slice;
+};
+
+// The CTA's i-th unit of work (all roles walk the same sequence).
+__device__ __forceinline__ bool next_work(const Params& p, int tiles, int i, Work& w) {
+    const int full = p.tail_split > 1 ? p.full_tiles : tiles;
+    const int t = blockIdx.x + i * gridDim.x;
+    if (t < full) {
+        w = {t, 0, p.nkb, -1};
+        return true;
+    }
+    if (p.tail_split > 1 && i == p.full_tiles / static_cast<int>(gridDim.x)) {
+        const int u = blockIdx.x;
+        if (u < (tiles - full) * p.tail_split) {
+            const int sl = u % p.tail_split;
+            w = {full + u / p.tail_split, sl * p.nkb / p.tail_split, (sl + 1) * p.nkb / p.tail_split, sl};
+            return true;
+        }
+    }
+    return false;
+}
+
+// Tile configuration.  The promotion warpgroups split the tile's columns.
+// BN = 192 uses three of them (64 columns per warp): every warp then reads its
+// whole share of a K block's partial in one TMEM round trip and hands the
+// buffer back before its FMAs, which keeps the FMAs off the path that frees
+// TMEM for the next MMA.  BN = 256 uses two (128 columns per warp, read in two
+// halves with FMAs in between -- accumulators plus a whole share would not fit
+// in the register file).
 template <int BN>
 struct Cfg {
     static_assert(BN % 64 == 0 && BN >= 64 && BN <= 256, "BN must be 64, 128, 192 or 256");
     static constexpr int kTileBBytes = BN * kBK;
     static constexpr int kNBuf = (BN <= 128) ? 4 : 2;
     static constexpr int kTmemCols = (kNBuf * BN <= 256) ? 256 : 512;
-    static constexpr int kColsPerWarp = BN / 2;        // two warpgroups split the columns
+    static constexpr int kEpiWGs = (BN == 192) ? 3 : 2;     // promotion warpgroups
+    static constexpr int kEpiWarpsC = 4 * kEpiWGs;
+    static constexpr int kThreadsC = 32 * (kFirstEpiWarp + kEpiWarpsC);
+    static constexpr int kColsPerWarp = BN / kEpiWGs;
     static constexpr int kChunks = kColsPerWarp / 32;  // tcgen05.ld 32x32b.x32 chunks
     static constexpr int kBatch = kChunks < 2 ? kChunks : 2;  // chunks loaded per wait
     static constexpr bool kSplitRegs = BN > 128;       // needs setmaxnreg rebalancing
+    // setmaxnreg budgets (multiples of 8) for the producer/MMA/scale warpgroup
+    // and the promotion warpgroups; their sum over all threads stays within
+    // the 64 K registers the CTA launches with.
+    static constexpr int kRegsLow = kEpiWGs == 3 ? 40 : 56;
+    static constexpr int kRegsHigh = kEpiWGs == 3 ? 152 : 224;
+    static_assert(128 * kRegsLow + 128 * kEpiWGs * kRegsHigh <= 65536, "register split exceeds the file");
     static_assert(kNBuf * BN <= kTmemCols, "TMEM buffers overflow the allocation");
     static_assert(kChunks % kBatch == 0, "chunk batching");
 };
@@ -81,7 +129,7 @@ template <int BN, int STAGES>
 constexpr int smem_bytes() {
     // 1 KiB alignment slack + operand ring + output staging + barriers and
     // bookkeeping (512 B) + scale ring + masked prefix table.
-    return 1024 + STAGES * (kTileABytes + Cfg<BN>::kTileBBytes) + kEpiWarps * kStageOutBytes + 512 +
+    return 1024 + STAGES * (kTileABytes + Cfg<BN>::kTileBBytes) + Cfg<BN>::kEpiWarpsC * kStageOutBytes + 512 +
            kScaleSlots * kScaleSlotFloats * 4 + 4 * (kMaxMaskedGroups + 1);
 }
 
@@ -136,7 +184,7 @@ __device__ __forceinline__ Tile decode_tile(const Params& p, int t, int m_blocks
 }
 
 template <int BN, int STAGES, int MODE>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(Cfg<BN>::kThreadsC, 1)
 fp8_gemm_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtensorMap tmA,
                 const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmD) {
     using C = Cfg<BN>;
@@ -147,7 +195,7 @@ fp8_gemm_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtens
     uint8_t* sA = smem;
     uint8_t* sB = sA + STAGES * kTileABytes;
     uint8_t* sOut = sB + STAGES * C::kTileBBytes;  // 1 KiB aligned, kStageOutBytes per promotion warp
-    uint64_t* full = reinterpret_cast<uint64_t*>(sOut + kEpiWarps * kStageOutBytes);
+    uint64_t* full = reinterpret_cast<uint64_t*>(sOut + C::kEpiWarpsC * kStageOutBytes);
     uint64_t* empty = full + STAGES;
     uint64_t* tfull = empty + STAGES;
     uint64_t* tempty = tfull + kNBuf;
@@ -169,11 +217,11 @@ fp8_gemm_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtens
         }
         for (int b = 0; b < kNBuf; ++b) {
             mbar_init(tfull + b, 1);
-            mbar_init(tempty + b, kEpiWarps);
+            mbar_init(tempty + b, C::kEpiWarpsC);
         }
         for (int s = 0; s < kScaleSlots; ++s) {
             mbar_init(sfull + s, 32);
-            mbar_init(sempty + s, kEpiWarps);
+            mbar_init(sempty + s, C::kEpiWarpsC);
         }
         mbar_init(done, 1);
         *abort_flag = 0;
@@ -193,7 +241,7 @@ fp8_gemm_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtens
         // Per-group m-block counts from the device-resident masked_m, then an
         // exclusive prefix over groups.  Counts outside [0, M_max] are clamped
         // and flagged.
-        for (int g = threadIdx.x; g < p.G; g += kThreads) {
+        for (int g = threadIdx.x; g < p.G; g += C::kThreadsC) {
             int mm = __ldg(p.masked_m + g);
             if (mm < 0 || mm > p.M) {
                 atomicOr(&g_dg_error, 4u);
@@ -230,7 +278,7 @@ fp8_gemm_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtens
     // the promotion warps hold BN/2 FP32 accumulators each.  Each branch sets
     // its own budget so that the compiler allocates every role against it.
     if (warp < kFirstEpiWarp) {
-    if (C::kSplitRegs) regs_dec<56>();
+    if (C::kSplitRegs) regs_dec<C::kRegsLow>();
     if (warp == 0) {
         // ------------------------------------------------------ producer ----
         const uint64_t pol_a = l2_policy_evict_last();
@@ -239,10 +287,11 @@ fp8_gemm_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtens
         uint32_t phase = 0;
         int fills = 0;
         bool ok = true;
-        for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
-            const Tile tl = decode_tile<BN, MODE>(p, t, m_blocks, mb_prefix);
+        Work w;
+        for (int it = 0; ok && next_work(p, tiles, it, w); ++it) {
+            const Tile tl = decode_tile<BN, MODE>(p, w.t, m_blocks, mb_prefix);
             if (!tl.valid) continue;
-            for (int kb = 0; kb < nkb; ++kb) {
+            for (int kb = w.kb0; kb < w.kb1; ++kb) {
                 if (!mbar_wait(empty + stage, phase ^ 1u, abort_flag)) { ok = false; break; }
                 if (lane == 0) {
                     mbar_arrive_expect_tx(full + stage, kTileABytes + C::kTileBBytes);
@@ -271,10 +320,11 @@ fp8_gemm_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtens
         int stage = 0, buf = 0;
         uint32_t phase = 0, bphase = 0;
         bool ok = true;
-        for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
-            const Tile tl = decode_tile<BN, MODE>(p, t, m_blocks, mb_prefix);
+        Work w;
+        for (int it = 0; ok && next_work(p, tiles, it, w); ++it) {
+            const Tile tl = decode_tile<BN, MODE>(p, w.t, m_blocks, mb_prefix);
             if (!tl.valid) continue;
-            for (int kb = 0; kb < nkb; ++kb) {
+            for (int kb = w.kb0; kb < w.kb1; ++kb) {
                 if (!mbar_wait(tempty + buf, bphase ^ 1u, abort_flag)) { ok = false; break; }
                 if (!mbar_wait(full + stage, phase, abort_flag)) { ok = false; break; }
                 tc_fence_after();
@@ -310,8 +360,9 @@ fp8_gemm_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtens
         int slot = 0;
         uint32_t sphase = 0;
         const int row_limit = p.M;  // rows of sa that exist (dense M, M_total or M_max)
-        for (int t = blockIdx.x; t < tiles; t += gridDim.x) {
-            const Tile tl = decode_tile<BN, MODE>(p, t, m_blocks, mb_prefix);
+        Work w;
+        for (int it = 0; next_work(p, tiles, it, w); ++it) {
+            const Tile tl = decode_tile<BN, MODE>(p, w.t, m_blocks, mb_prefix);
             if (!tl.valid) continue;
             const float* sa_base = p.sa + (MODE == kMasked ? static_cast<int64_t>(tl.g) * nkb * p.sa_stride : 0);
             const float* sb_g = p.sb + static_cast<int64_t>(tl.g) * p.nbn * nkb;
@@ -321,7 +372,7 @@ fp8_gemm_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtens
             const int left = row_limit - r4;
             const uint32_t sa_bytes = left >= 4 ? 16u : (left > 0 ? static_cast<uint32_t>(left) * 4u : 0u);
             bool ok = true;
-            for (int kb = 0; kb < nkb; ++kb) {
+            for (int kb = w.kb0; kb < w.kb1; ++kb) {
                 if (!mbar_wait(sempty + slot, sphase ^ 1u, abort_flag)) { ok = false; break; }
                 const uint32_t dst = smem_u32(sring + slot * kScaleSlotFloats);
                 const float* src = sa_bytes ? sa_base + static_cast<int64_t>(kb) * p.sa_stride + r4 : p.sa;
@@ -339,9 +390,9 @@ fp8_gemm_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtens
     }
     } else {
         // ------------------------------------------ promotion + epilogue ----
-        if (C::kSplitRegs) regs_inc<224>();
+        if (C::kSplitRegs) regs_inc<C::kRegsHigh>();
         const int ew = warp - kFirstEpiWarp;
-        const int half = ew >> 2;                 // which half of the tile's columns
+        const int half = ew >> 2;                 // which warpgroup's share of the tile's columns
         const int quarter = warp & 3;             // TMEM lane quarter this warp may access
         const int r = quarter * 32 + lane;        // row inside the tile
         const int col0 = half * C::kColsPerWarp;  // first column inside the tile
@@ -349,8 +400,9 @@ fp8_gemm_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtens
         int buf = 0, slot = 0;
         uint32_t bphase = 0, sphase = 0;
         bool ok = true;
-        for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
-            const Tile tl = decode_tile<BN, MODE>(p, t, m_blocks, mb_prefix);
+        Work w;
+        for (int it = 0; ok && next_work(p, tiles, it, w); ++it) {
+            const Tile tl = decode_tile<BN, MODE>(p, w.t, m_blocks, mb_prefix);
             if (!tl.valid) continue;
             const int g = tl.g;
             // Row validity and the row's output address.
@@ -379,7 +431,7 @@ fp8_gemm_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtens
 #pragma unroll
             for (int j = 0; j < C::kColsPerWarp / 2; ++j) acc[j] = make_float2(0.f, 0.f);
 
-            for (int kb = 0; kb < nkb; ++kb) {
+            for (int kb = w.kb0; kb < w.kb1; ++kb) {
                 if (!mbar_wait(sfull + slot, sphase, abort_flag)) { ok = false; break; }
                 const float* sc = sring + slot * kScaleSlotFloats;
                 const float s_a = sc[r];
@@ -421,6 +473,53 @@ fp8_gemm_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtens
                 if (++buf == kNBuf) { buf = 0; bphase ^= 1u; }
             }
             if (!ok) break;
+
+            if (w.slice >= 0) {
+                // Split tail tile.  Partial (r, s) for slices s >= 1 lives at
+                // ws + ((r*(S-1) + s-1) * 128*BN) floats in the layout
+                // [promotion warp][float4 j][lane], so a warp moves 512
+                // contiguous bytes per access.  Slice s >= 1 writes its partial
+                // and raises its flag; slice 0 waits for every flag, adds the
+                // partials in slice order (fixed, so the result is
+                // deterministic), resets the flags and stores D.
+                constexpr int kF4 = C::kColsPerWarp / 4;
+                const int S = p.tail_split;
+                const int rt = w.t - p.full_tiles;
+                const int nthreads = 32 * C::kEpiWarpsC;
+                const bool leader = (warp == kFirstEpiWarp && lane == 0);
+                if (w.slice > 0) {
+                    float4* dst = reinterpret_cast<float4*>(p.ws + static_cast<int64_t>(rt * (S - 1) + w.slice - 1) * kBM * BN);
+#pragma unroll
+                    for (int j = 0; j < kF4; ++j)
+                        __stcg(dst + (ew * kF4 + j) * 32 + lane,
+                               make_float4(acc[2 * j].x, acc[2 * j].y, acc[2 * j + 1].x, acc[2 * j + 1].y));
+                    __threadfence();
+                    named_barrier_sync(1, nthreads);
+                    if (leader) st_release_gpu(p.ws_flags + rt * (S - 1) + w.slice - 1, 1u);
+                    continue;  // slice 0 stores the tile
+                }
+                // slice 0
+                bool got = true;
+                if (leader) {
+                    for (int s2 = 1; s2 < S && got; ++s2)
+                        got = wait_flag_gpu(p.ws_flags + rt * (S - 1) + s2 - 1);
+                    for (int s2 = 1; s2 < S; ++s2) p.ws_flags[rt * (S - 1) + s2 - 1] = 0u;
+                    if (!got) atomicOr(&g_dg_error, 1u);
+                }
+                named_barrier_sync(1, nthreads);
+                for (int s2 = 1; s2 < S; ++s2) {
+                    const float4* src = reinterpret_cast<const float4*>(
+                        p.ws + static_cast<int64_t>(rt * (S - 1) + s2 - 1) * kBM * BN);
+#pragma unroll
+                    for (int j = 0; j < kF4; ++j) {
+                        const float4 v = __ldcg(src + (ew * kF4 + j) * 32 + lane);
+                        acc[2 * j].x += v.x;
+                        acc[2 * j].y += v.y;
+                        acc[2 * j + 1].x += v.z;
+                        acc[2 * j + 1].y += v.w;
+                    }
+                }
+            }
 
             // Epilogue: bf16 round-to-nearest-even.  When every row of this
             // warp may be written (valid, or outside D where the TMA store

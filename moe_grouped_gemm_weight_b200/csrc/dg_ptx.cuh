@@ -61,6 +61,24 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     return ok != 0;
 }
 
+// try_wait with a suspend-time hint: the thread is parked (not polling) until
+// the phase completes or about `hint_ns` pass, whichever comes first.
+__device__ __forceinline__ bool mbar_try_wait_hint(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return ok != 0;
+}
+
+// Suspend hint of the blocking waits: long enough that a waiting warp stays
+// parked until its barrier completes, short enough to notice an abort.
+constexpr uint32_t kWaitHintNs = 1000000;  // 1 ms
+
 // Wait until the phase with the given parity has completed.  Gives up (and
 // raises *abort_flag plus the TIMEOUT error bit) after kWaitLimitNs, or at
 // once when another role has already raised *abort_flag.
@@ -68,7 +86,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     while (true) {
-        if (mbar_try_wait(bar, parity)) return true;
+        if (mbar_try_wait_hint(bar, parity, kWaitHintNs)) return true;
         if (*abort_flag) return false;
         if (globaltimer_ns() - t0 > kWaitLimitNs) {
             *abort_flag = 1;
@@ -81,7 +99,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
 // Clean-up wait: ignores the abort flag, bounded by kDrainLimitNs.
 __device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity) {
     const uint64_t t0 = globaltimer_ns();
-    while (!mbar_try_wait(bar, parity)) {
+    while (!mbar_try_wait_hint(bar, parity, kWaitHintNs)) {
         if (globaltimer_ns() - t0 > kDrainLimitNs) {
             atomicOr(&g_dg_error, 1u);
             return false;
@@ -182,6 +200,34 @@ __device__ __forceinline__ float4 ld_nc_f4(const float* p) {
                  : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
                  : "l"(p));
     return v;
+}
+
+// ----------------------------------------------------- grid-level flags ----
+
+// Barrier over `count` threads of the CTA (named barrier `id`, not 0).
+__device__ __forceinline__ void named_barrier_sync(int id, int count) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void st_release_gpu(unsigned int* p, unsigned int v) {
+    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ unsigned int ld_acquire_gpu(const unsigned int* p) {
+    unsigned int v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// Wait (bounded by kWaitLimitNs) until another CTA sets *flag != 0.
+__device__ __forceinline__ bool wait_flag_gpu(const unsigned int* flag) {
+    if (ld_acquire_gpu(flag)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    while (!ld_acquire_gpu(flag)) {
+        if (globaltimer_ns() - t0 > kWaitLimitNs) return false;
+        __nanosleep(64);
+    }
+    return true;
 }
 
 // ------------------------------------------------ asynchronous small copies ----

@@ -324,3 +324,23 @@ def test_pair_kernel_masked_full(dgm, force_pair):
     for g in range(4):
         assert_close(got[g, :mm[g]], ref[g, :mm[g]], mag[g, :mm[g]], f"pair masked g={g}")
     assert dgm.dg_get_device_error() == 0
+
+
+# ------------------------------------------- K-split of the last partial wave --
+
+@pytest.mark.parametrize("M,N,K,sms,split", [(256, 1536, 4096, 5, 2), (384, 1792, 6144, 20, 3),
+                                             (384, 1792, 8192, 20, 4)])
+def test_tail_split_matches_oracle_and_is_deterministic(dgm, M, N, K, sms, split):
+    c = wl.dense_case(M, N, K, seed=M + N + K + sms)
+    try:
+        dgm.dg_set_num_sms(sms)
+        plan = dgm.dg_make_plan(0, M, N, K, 1, sms)
+        assert plan["tail_split"] == split and plan["tiles"] % plan["grid"] != 0
+        a = run_dense(dgm, c)
+        b = run_dense(dgm, c)
+    finally:
+        dgm.dg_set_num_sms(0)
+    assert np.array_equal(a, b)
+    ref, mag = oracle_dense(c)
+    assert_close(a, ref, mag, f"tail split {split}")
+    assert dgm.dg_get_device_error() == 0
