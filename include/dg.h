@@ -94,6 +94,29 @@ DG_API dg_status dg_fp8_gemm_nt(uint16_t* D, const uint8_t* A, const float* sa, 
                          const uint8_t* B, const float* sb, int M, int N, int K, void* stream);
 
 /*
+ * Dense GEMM that allocates nothing.  The pages describe no such call; it
+ * exists for callers that must not allocate device memory once they are
+ * running: a serving loop that reserved all of HBM for its own pool up front,
+ * or code that cannot afford the device-wide synchronisation cudaMalloc and
+ * cudaFree may bring.  Same arguments, layouts and result as dg_fp8_gemm_nt.
+ *
+ * Where the last wave of tiles is split along K, its FP32 partials and flags
+ * live in one static device array of 16 MiB + 4 KiB, held on every GPU that
+ * loads the library until the process exits, instead of in a workspace the
+ * library allocates.  A call whose split would need more than that returns
+ * DG_ERR_UNSUPPORTED and launches nothing (on a 148-SM B200 no call does).
+ * The flags are cleared on the stream before each launch that uses them.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture starts.
+ *   - Every call on a device shares the one array: calls that may overlap on
+ *     the GPU (other streams, or a concurrent thread) race on it and give
+ *     wrong results.  Order them on one stream or with events.
+ */
+DG_API dg_status dg_fp8_gemm_nt_noalloc(uint16_t* D, const uint8_t* A, const float* sa, int sa_stride,
+                                        const uint8_t* B, const float* sb, int M, int N, int K, void* stream);
+
+/*
  * Grouped GEMM, contiguous layout (section "分组 GEMM（连续布局）"): the rows of
  * all groups are concatenated along M and share N and K.  m_indices[m] (int32,
  * device) is the group of row m; -1 marks a padding row, whose D row is left

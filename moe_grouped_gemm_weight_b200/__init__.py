@@ -56,6 +56,8 @@ def lib() -> ctypes.CDLL:
             P, I = ctypes.c_void_p, ctypes.c_int
             L.dg_fp8_gemm_nt.restype = I
             L.dg_fp8_gemm_nt.argtypes = [P, P, P, I, P, P, I, I, I, P]
+            L.dg_fp8_gemm_nt_noalloc.restype = I
+            L.dg_fp8_gemm_nt_noalloc.argtypes = [P, P, P, I, P, P, I, I, I, P]
             L.dg_grouped_contiguous_nt.restype = I
             L.dg_grouped_contiguous_nt.argtypes = [P, P, P, I, P, P, P, I, I, I, I, P]
             L.dg_grouped_masked_nt.restype = I
@@ -106,6 +108,17 @@ def dg_fp8_gemm_nt(D, A, sa, sa_stride: int, B, sb, stream=None) -> None:
     N = B.shape[-2]
     _check("dg_fp8_gemm_nt", lib().dg_fp8_gemm_nt(_ptr(D), _ptr(A), _ptr(sa), int(sa_stride), _ptr(B), _ptr(sb),
                                                   M, N, K, _stream(stream)))
+
+
+def dg_fp8_gemm_nt_noalloc(D, A, sa, sa_stride: int, B, sb, stream=None) -> None:
+    """dg_fp8_gemm_nt without device allocation: the K-split scratch is a static
+    16 MiB array shared by every call on the device, so calls that overlap on
+    the GPU race.  Make the first call on each device before any stream capture."""
+    M, K = A.shape[-2], A.shape[-1]
+    N = B.shape[-2]
+    _check("dg_fp8_gemm_nt_noalloc",
+           lib().dg_fp8_gemm_nt_noalloc(_ptr(D), _ptr(A), _ptr(sa), int(sa_stride), _ptr(B), _ptr(sb),
+                                        M, N, K, _stream(stream)))
 
 
 def dg_grouped_contiguous_nt(D, A, sa, sa_stride: int, B, sb, m_indices, stream=None) -> None:

@@ -601,6 +601,49 @@ dg::Params make_params(uint16_t* D, const float* sa, int sa_stride, const float*
 
 }  // namespace
 
+// ------------------------------------------------ allocation-free dense ----
+// dg_fp8_gemm_nt_noalloc keeps the K-split tail's scratch in this fixed
+// array instead of a workspace from cudaMalloc: FP32 partials in the first
+// 16 MiB (128 tiles of 128 x 256), then 1024 ready flags.  The array is zero
+// at module load and every GPU that loads the library holds it until the
+// process exits.  All calls on a GPU share it.
+constexpr size_t kNoAllocPartialBytes = size_t(16) << 20;
+constexpr size_t kNoAllocFlags = 1024;
+static __device__ __align__(256) unsigned char dg_noalloc_scratch[kNoAllocPartialBytes +
+                                                                  kNoAllocFlags * sizeof(unsigned int)];
+
+namespace {
+
+// Device address of dg_noalloc_scratch on the current device.  On the host the
+// symbol is only a handle, so the address is looked up once per device (with
+// that device current) and cached.
+dg_status noalloc_scratch(unsigned char** out) {
+    static std::mutex mu;
+    static std::map<int, unsigned char*> addrs;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return fail(DG_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+    }
+    std::lock_guard<std::mutex> lock(mu);
+    auto it = addrs.find(dev);
+    if (it == addrs.end()) {
+        unsigned char* ptr = nullptr;
+        e = cudaGetSymbolAddress((void**)&ptr, dg_noalloc_scratch);
+        if (e != cudaSuccess || ptr == nullptr) {
+            cudaGetLastError();
+            return fail(DG_ERR_CUDA, "cudaGetSymbolAddress(dg_noalloc_scratch) on device %d: %s", dev,
+                        cudaGetErrorString(e));
+        }
+        it = addrs.emplace(dev, ptr).first;
+    }
+    *out = it->second;
+    return DG_OK;
+}
+
+}  // namespace
+
 extern "C" {
 
 dg_status dg_fp8_gemm_nt(uint16_t* D, const uint8_t* A, const float* sa, int sa_stride, const uint8_t* B,
@@ -635,6 +678,59 @@ dg_status dg_fp8_gemm_nt(uint16_t* D, const uint8_t* A, const float* sa, int sa_
         p.ws_flags = ws.flags;
     }
     return dispatch<dg::kDense>(pl, p, ta, tb, td, static_cast<cudaStream_t>(stream));
+}
+
+dg_status dg_fp8_gemm_nt_noalloc(uint16_t* D, const uint8_t* A, const float* sa, int sa_stride, const uint8_t* B,
+                                 const float* sb, int M, int N, int K, void* stream) {
+    dg_status s = check_sizes(0, M, N, K, 1);
+    if (s != DG_OK) return s;
+    if ((s = common_checks(D, A, sa, sa_stride, B, sb, M)) != DG_OK) return s;
+    if (M == 0) return ok();
+    unsigned char* scratch = nullptr;
+    if ((s = noalloc_scratch(&scratch)) != DG_OK) return s;
+    const int sms = effective_sms();
+    if (sms <= 0) return fail(DG_ERR_CUDA, "no CUDA device");
+    dg_plan pl;
+    if ((s = plan(0, M, N, K, 1, sms, &pl)) != DG_OK) return s;
+    const cudaStream_t st = static_cast<cudaStream_t>(stream);
+    CUtensorMap ta, tb;
+    if (pl.swap_ab) {
+        if ((s = make_operand_map(&ta, A, K, M, 1, pl.block_m, false)) != DG_OK) return s;
+        if ((s = make_operand_map(&tb, B, K, N, 1, 128, true)) != DG_OK) return s;
+        dg::Params p = make_params(D, sa, sa_stride, sb, M, N, K, 1, pl);
+        return dispatch_small<dg::kDense>(pl, p, ta, tb, st);
+    }
+    if ((s = make_operand_map(&ta, A, K, M, 1, dg::kBM, false)) != DG_OK) return s;
+    if ((s = make_operand_map(&tb, B, K, N, 1, pl.cta_pair ? pl.block_n / 2 : pl.block_n, true)) != DG_OK) return s;
+    CUtensorMap td;
+    if ((s = make_output_map(&td, D, N, M, 1, false)) != DG_OK) return s;
+    dg::Params p = make_params(D, sa, sa_stride, sb, M, N, K, 1, pl);
+    p.b_stream = pl.m_blocks == 1;
+    if (pl.cta_pair) return launch_pair<dg::kDense>(p, ta, tb, td, pl, st);
+    if (pl.tail_split > 1) {
+        // One partial per (tail tile, slice >= 1) and one flag per partial.
+        const int full = (pl.tiles / pl.grid) * pl.grid;
+        const size_t slots = static_cast<size_t>(pl.tiles - full) * (pl.tail_split - 1);
+        const size_t part_bytes = slots * dg::kBM * pl.block_n * sizeof(float);
+        if (part_bytes > kNoAllocPartialBytes || slots > kNoAllocFlags)
+            return fail(DG_ERR_UNSUPPORTED,
+                        "dg_fp8_gemm_nt_noalloc: M=%d N=%d K=%d on %d SMs needs %zu bytes of K-split partials "
+                        "and %zu flags; the static scratch holds %zu bytes and %zu flags",
+                        M, N, K, pl.grid, part_bytes, slots, kNoAllocPartialBytes, kNoAllocFlags);
+        unsigned int* flags = reinterpret_cast<unsigned int*>(scratch + kNoAllocPartialBytes);
+        // The flags must start at zero; a previous call that gave up on a wait
+        // may have left some set.  The partials are always written before read.
+        const cudaError_t e = cudaMemsetAsync(flags, 0, slots * sizeof(unsigned int), st);
+        if (e != cudaSuccess) {
+            cudaGetLastError();
+            return fail(DG_ERR_CUDA, "clearing the scratch flags: %s", cudaGetErrorString(e));
+        }
+        p.tail_split = pl.tail_split;
+        p.full_tiles = full;
+        p.ws = reinterpret_cast<float*>(scratch);
+        p.ws_flags = flags;
+    }
+    return dispatch<dg::kDense>(pl, p, ta, tb, td, st);
 }
 
 dg_status dg_grouped_contiguous_nt(uint16_t* D, const uint8_t* A, const float* sa, int sa_stride, const uint8_t* B,
