@@ -1,7 +1,8 @@
 // dg_api.cu -- host side of the C ABI declared in include/dg.h: argument
 // validation, the launch plan (tile shape, ring depth, grid), TMA tensor-map
-// encoding and kernel dispatch.  Nothing here allocates device memory, reads
-// device memory or synchronises, except dg_get_device_error().
+// encoding and kernel dispatch.  Nothing here reads device memory or
+// synchronises, except dg_get_device_error(); the only device allocation is
+// the per-(device, stream) K-split workspace, made once on first need.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
