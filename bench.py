@@ -9,8 +9,9 @@ scales, bf16 output -- 18 GEMMs through the C ABI.  Inputs are larger than L2:
 each shape cycles over enough copies of its operands (>= 3 x the 126 MB L2 in
 total) that every launch reads operands last touched at least 3 x L2 of other
 traffic ago.  The K launches of each shape are captured in one CUDA graph and
-timed with CUDA events around its replay on the capture stream, so host launch
-overhead stays out of microsecond-scale decode shapes.  ``value`` is the
+timed with CUDA events around its replay on the capture stream (after one
+untimed replay that uploads the graph), so host launch overhead stays out of
+microsecond-scale decode shapes.  ``value`` is the
 aggregate TFLOP/s of the sweep (sum of flops / sum of kernel times), max over
 ranks for N > 1 (each rank runs the same sweep on its own GPU: weak scaling, no
 collective on the data path).  Per shape, ``us_flushed`` is also given: a
@@ -275,6 +276,11 @@ class RotatingGraph:
                 rc, rd = self.reps[i % self.copies]
                 p.run(case=rc, D=rd)
         self.ev = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+        # The first replay of a graph also uploads it (about 2 us per launch
+        # for microsecond kernels): do it untimed.
+        with torch.cuda.stream(stream):
+            self.graph.replay()
+        stream.synchronize()
 
     def replay(self):
         # CUDAGraph.replay launches on the current stream: make it the one the

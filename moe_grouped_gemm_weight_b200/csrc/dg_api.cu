@@ -348,6 +348,24 @@ dg_status plan(int mode, int rows, int N, int K, int G, int num_sms, dg_plan* ou
 
 // ------------------------------------------------------------ launch ----
 
+// With DG_PDL=1 every GEMM launch allows programmatic dependent launch: the
+// kernel's set-up (barriers, TMEM, tensor-map and weight prefetch) may overlap
+// the end of the previous kernel in the stream; the kernels always wait
+// (griddepcontrol.wait) before touching global data.  It is off by default:
+// measured in CUDA-graph replays it shortens some decode-sized launches (e.g.
+// 64x32768x512 by about a quarter) but lengthens cluster launches with large
+// grids (64x7168x16384 by up to a third), whose CTAs are then placed into
+// slots as the previous grid frees them instead of spread over an idle GPU.
+bool pdl_enabled() {
+    const char* v = std::getenv("DG_PDL");
+    return v && v[0] == '1';
+}
+
+void set_pdl(cudaLaunchAttribute& a) {
+    a.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    a.val.programmaticStreamSerializationAllowed = pdl_enabled() ? 1 : 0;
+}
+
 template <int BN, int STAGES, int MODE>
 dg_status launch_one(const dg::Params& p, const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& td,
                      int grid, cudaStream_t stream) {
@@ -362,8 +380,17 @@ dg_status launch_one(const dg::Params& p, const CUtensorMap& ta, const CUtensorM
             return fail(DG_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(cudaGetLastError()));
         attr_set[dev].store(1);
     }
-    kern<<<grid, dg::Cfg<BN>::kThreadsC, smem, stream>>>(p, ta, tb, td);
-    cudaError_t e = cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
+    cfg.blockDim = dim3(dg::Cfg<BN>::kThreadsC, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    set_pdl(attr[0]);
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kern, p, ta, tb, td);
+    if (e == cudaSuccess) e = cudaGetLastError();
     if (e != cudaSuccess) return fail(DG_ERR_CUDA, "kernel launch failed: %s", cudaGetErrorString(e));
     return ok();
 }
@@ -426,13 +453,14 @@ dg_status launch_pair(const dg::Params& p, const CUtensorMap& ta, const CUtensor
     cfg.blockDim = dim3(dg::kThreads, 1, 1);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = 2;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    set_pdl(attr[1]);
+    cfg.numAttrs = 2;
     cudaError_t e = cudaLaunchKernelEx(&cfg, kern, p, ta, tb, td);
     if (e == cudaSuccess) e = cudaGetLastError();
     if (e != cudaSuccess) return fail(DG_ERR_CUDA, "kernel launch failed: %s", cudaGetErrorString(e));
@@ -459,13 +487,14 @@ dg_status launch_small(const dg::Params& p, const CUtensorMap& ta, const CUtenso
     cfg.blockDim = dim3(dg::kSmallThreads, 1, 1);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = static_cast<unsigned>(pl.split_k);
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    set_pdl(attr[1]);
+    cfg.numAttrs = 2;
     cudaError_t e = cudaLaunchKernelEx(&cfg, kern, p, ta, tb);
     if (e == cudaSuccess) e = cudaGetLastError();
     if (e != cudaSuccess) return fail(DG_ERR_CUDA, "kernel launch failed: %s", cudaGetErrorString(e));

@@ -236,6 +236,10 @@ fp8_gemm_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtens
         tmem_alloc(tmem_slot, C::kTmemCols);
         tmem_relinquish();
     }
+    // Nothing above reads or writes global data: with programmatic dependent
+    // launch it overlaps the end of the previous kernel in the stream.
+    griddep_wait();
+    griddep_launch_dependents();
     int m_blocks = p.m_blocks;
     if (MODE == kMasked) {
         // Per-group m-block counts from the device-resident masked_m, then an

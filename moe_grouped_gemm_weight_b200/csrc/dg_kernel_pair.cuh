@@ -133,6 +133,9 @@ fp8_gemm_pair_kernel(const __grid_constant__ Params p, const __grid_constant__ C
         tmem_alloc_pair(tmem_slot, C::kTmemCols);
         tmem_relinquish_pair();
     }
+    // Nothing above reads or writes global data (see the single-CTA kernel).
+    griddep_wait();
+    griddep_launch_dependents();
     int m_blocks = p.m_blocks;
     if (MODE == kMasked) {
         for (int g = threadIdx.x; g < p.G; g += kThreads) {

@@ -73,6 +73,8 @@ fp8_gemm_swapab_kernel(const __grid_constant__ Params p, const __grid_constant__
     }
     int rows_valid = p.M;
     if (MODE == kMasked) {
+        // masked_m may come from the previous kernel in the stream.
+        griddep_wait();
         const int mm = __ldg(p.masked_m + g);
         if ((mm < 0 || mm > p.M) && rank == 0 && blockIdx.y == 0 && m0 == 0) atomicOr(&g_dg_error, 4u);
         rows_valid = min(max(mm, 0), p.M);
@@ -132,16 +134,22 @@ fp8_gemm_swapab_kernel(const __grid_constant__ Params p, const __grid_constant__
         mbar_init(done, 1);
         *abort_flag = 0;
         fence_mbar_init();
-        // The ring starts empty: issue its first loads now, so that their
-        // latency overlaps the rest of the set-up.
+        // The ring starts empty: pull its first weight tiles into L2 while the
+        // previous kernel may still run, then (once its data is visible)
+        // issue the first loads, so that their latency overlaps the rest of
+        // the set-up.
         prefetch_tmap(&tmA);
         prefetch_tmap(&tmB);
+        for (int i = 0; i < STAGES && kb0 + i < kb1; ++i) tma_prefetch_3d(&tmB, (kb0 + i) * kBK, n0, g);
+        griddep_wait();
         for (int i = 0; i < STAGES && kb0 + i < kb1; ++i) issue_stage(i, kb0 + i);
     }
     if (warp == 1) {
         tmem_alloc(tmem_slot, kSmallTmemCols);
         tmem_relinquish();
     }
+    griddep_wait();
+    griddep_launch_dependents();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();

@@ -202,6 +202,30 @@ __device__ __forceinline__ float4 ld_nc_f4(const float* p) {
     return v;
 }
 
+// ------------------------------------- programmatic dependent launch ----
+// A kernel launched with programmatic stream serialization (opt-in, see the
+// launch code) may start while the previous kernel in the stream is still
+// finishing.  griddep_wait()
+// blocks the calling thread until that kernel has completed and its memory
+// is visible; every thread calls it before touching global data another
+// kernel may have written.  griddep_launch_dependents() lets the next such
+// kernel start its own set-up early (without the launch attribute both are
+// no-ops).
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Prefetch of one TMA box into L2 (no shared memory, no barrier).  L2 is the
+// point of coherence, so a prefetch issued before griddep_wait() can never
+// make a later read return data older than the wait exposes.
+__device__ __forceinline__ void tma_prefetch_3d(const CUtensorMap* tm, int x, int y, int z) {
+    asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(
+                     reinterpret_cast<uint64_t>(tm)),
+                 "r"(x), "r"(y), "r"(z)
+                 : "memory");
+}
+
 // ----------------------------------------------------- grid-level flags ----
 
 // Barrier over `count` threads of the CTA (named barrier `id`, not 0).

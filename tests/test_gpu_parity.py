@@ -344,3 +344,85 @@ def test_tail_split_matches_oracle_and_is_deterministic(dgm, M, N, K, sms, split
     ref, mag = oracle_dense(c)
     assert_close(a, ref, mag, f"tail split {split}")
     assert dgm.dg_get_device_error() == 0
+
+
+# ------------------------------------- back-to-back launches (PDL) --------
+# With DG_PDL=1 GEMM launches allow programmatic dependent launch: a kernel may
+# start its set-up while the previous kernel in the stream finishes.  It must
+# still read the inputs that kernel wrote, write D after it, and use the
+# K-split workspace only after it.  Each test runs with PDL on and off.
+
+@pytest.fixture(params=["pdl", "serial"])
+def pdl_mode(request, monkeypatch):
+    monkeypatch.setenv("DG_PDL", "1" if request.param == "pdl" else "0")
+    yield request.param
+
+def _fill_from(dst: wl.Case, src: wl.Case):
+    for k in ("A", "sa", "B", "sb"):
+        getattr(dst, k).copy_(getattr(src, k))
+
+
+@pytest.mark.parametrize("M,N,K", [(64, 2112, 1024), (4096, 1024, 1024)])
+def test_inputs_written_just_before_the_gemm_are_seen(dgm, pdl_mode, M, N, K):
+    c1, c2 = wl.dense_case(M, N, K, seed=11), wl.dense_case(M, N, K, seed=12)
+    g1, g2 = c1.to("cuda"), c2.to("cuda")
+    work = wl.dense_case(M, N, K, seed=13).to("cuda")  # operand buffers rewritten before each call
+    D = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+    for _ in range(3):  # no synchronisation between the kernels
+        _fill_from(work, g1)
+        dgm.dg_fp8_gemm_nt(D, work.A, work.sa, work.sa_stride, work.B, work.sb)
+        _fill_from(work, g2)
+        dgm.dg_fp8_gemm_nt(D, work.A, work.sa, work.sa_stride, work.B, work.sb)
+    torch.cuda.synchronize()
+    rows = sample_rows(M, n_random=8, seed=4)
+    ref, mag = oracle_dense(c2, rows=rows)
+    assert_close(_bits(D)[rows], ref[rows], mag[rows], f"last of back-to-back GEMMs {M}x{N}x{K}")
+
+
+def test_back_to_back_k_split_gemms_share_the_workspace(dgm, pdl_mode):
+    # Tail-split launches back to back on one stream (distinct inputs and
+    # outputs): each publishes partials to the same workspace only after the
+    # previous launch has finished with it.
+    M, N, K, sms = 384, 1792, 8192, 20
+    cases = [wl.dense_case(M, N, K, seed=40 + i) for i in range(3)]
+    gs = [c.to("cuda") for c in cases]
+    Ds = [torch.empty(M, N, dtype=torch.bfloat16, device="cuda") for _ in cases]
+    try:
+        dgm.dg_set_num_sms(sms)
+        assert dgm.dg_make_plan(0, M, N, K, 1, sms)["tail_split"] > 1
+        for _ in range(2):
+            for g, D in zip(gs, Ds):
+                dgm.dg_fp8_gemm_nt(D, g.A, g.sa, g.sa_stride, g.B, g.sb)
+        torch.cuda.synchronize()
+    finally:
+        dgm.dg_set_num_sms(0)
+    for c, D in zip(cases, Ds):
+        ref, mag = oracle_dense(c)
+        assert_close(_bits(D), ref, mag, "back-to-back tail split")
+    assert dgm.dg_get_device_error() == 0
+
+
+def test_back_to_back_launches_in_a_cuda_graph(dgm, pdl_mode):
+    M, N, K = 64, 2112, 1024
+    c1, c2 = wl.dense_case(M, N, K, seed=21), wl.dense_case(M, N, K, seed=22)
+    g1, g2 = c1.to("cuda"), c2.to("cuda")
+    work = wl.dense_case(M, N, K, seed=23).to("cuda")
+    D1 = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+    D2 = torch.empty_like(D1)
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        dgm.dg_fp8_gemm_nt(D1, work.A, work.sa, work.sa_stride, work.B, work.sb)  # first call on s
+    s.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=s):
+        _fill_from(work, g1)
+        dgm.dg_fp8_gemm_nt(D1, work.A, work.sa, work.sa_stride, work.B, work.sb)
+        _fill_from(work, g2)
+        dgm.dg_fp8_gemm_nt(D2, work.A, work.sa, work.sa_stride, work.B, work.sb)
+    for _ in range(2):
+        with torch.cuda.stream(s):
+            graph.replay()
+    torch.cuda.synchronize()
+    for c, D in ((c1, D1), (c2, D2)):
+        ref, mag = oracle_dense(c)
+        assert_close(_bits(D), ref, mag, "graph back-to-back")
