@@ -71,6 +71,13 @@ def _load():
             lib.dgo_grouped_masked.restype = I
             lib.dgo_grouped_masked.argtypes = [P, P, I64, P, P, P, I, I, I, I, P, I64, P, P, P]
             lib.dgo_num_threads.restype = I
+            lib.dgo_e4m3_encode.restype = ctypes.c_uint8
+            lib.dgo_e4m3_encode.argtypes = [ctypes.c_float]
+            lib.dgo_e4m3_encode_array.argtypes = [P, P, I64]
+            lib.dgo_cast_1x128.restype = I
+            lib.dgo_cast_1x128.argtypes = [P, I, I, P, P, I64]
+            lib.dgo_cast_128x128.restype = I
+            lib.dgo_cast_128x128.argtypes = [P, I, I, P, P]
             _lib = lib
     return _lib
 
@@ -181,3 +188,34 @@ def grouped_masked(A, sa, sa_stride, B, sb, masked_m, G, Mmax, N, K, rows=None, 
     if rc != OK:
         raise ValueError(f"oracle grouped_masked rejected its arguments (code {rc})")
     return D, D64, MAG
+
+
+def e4m3_encode(x) -> np.ndarray:
+    """e4m3 codes (uint8) of float32 values: RNE, saturating to +-448, NaN -> 0x7F."""
+    x = _c(np.atleast_1d(np.asarray(x, dtype=np.float32)), np.float32)
+    out = np.empty(x.shape, dtype=np.uint8)
+    _load().dgo_e4m3_encode_array(_ptr(x), _ptr(out), x.size)
+    return out
+
+
+def cast_1x128(X_bf16, M, K, sa_stride):
+    """Activation cast: bf16 bits [M,K] -> (e4m3 codes [M,K], sa float32 flat with
+    sa[kb*sa_stride + m])."""
+    X = _c(X_bf16, np.uint16)
+    Q = np.zeros((M, K), dtype=np.uint8)
+    sa = np.zeros((K // 128) * sa_stride, dtype=np.float32)
+    rc = _load().dgo_cast_1x128(_ptr(X), M, K, _ptr(Q), _ptr(sa), sa_stride)
+    if rc != OK:
+        raise ValueError(f"oracle cast_1x128 rejected its arguments (code {rc})")
+    return Q, sa
+
+
+def cast_128x128(W_bf16, N, K):
+    """Weight cast: bf16 bits [N,K] -> (e4m3 codes [N,K], sb float32 [ceil(N/128), K/128])."""
+    W = _c(W_bf16, np.uint16)
+    Q = np.zeros((N, K), dtype=np.uint8)
+    sb = np.zeros(((N + 127) // 128, K // 128), dtype=np.float32)
+    rc = _load().dgo_cast_128x128(_ptr(W), N, K, _ptr(Q), _ptr(sb))
+    if rc != OK:
+        raise ValueError(f"oracle cast_128x128 rejected its arguments (code {rc})")
+    return Q, sb

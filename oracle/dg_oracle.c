@@ -273,3 +273,103 @@ int dgo_num_threads(void) { return omp_get_max_threads(); }
 #else
 int dgo_num_threads(void) { return 1; }
 #endif
+
+/* ------------------------------------------------------- FP8 cast ---- */
+/*
+ * The cast that produces the GEMM's FP8 operands and their scales.  The pages
+ * leave it to the caller: "DeepGEMM项目介绍与本地部署指南", section "接口"
+ * (Interface), asks for e4m3 inputs with transposed, TMA-aligned LHS scales;
+ * the later-version article (yfxerp.com), section 4.1, calls a helper
+ * to_fp8 that returns the FP8 tensor and its scale factors; the page "Deepseek
+ * DeepGEMM 技术原理的深入分析", section "技术背景与核心原理", fixes one scale
+ * per 1x128 activation tile and per 128x128 weight block.  Reading taken here,
+ * every step in IEEE single precision (the kernel takes each decision in the
+ * same precision, so the codes compare bit for bit):
+ *
+ *   amax = max(max over the tile of |x|, 1e-4)   (fmaxf: a NaN is skipped)
+ *   s    = amax / 448            the stored scale (sa or sb)
+ *   r    = 448 / amax
+ *   q    = e4m3_rne_satfinite(x * r)
+ *
+ * so that s * decode(q) ~ x and the largest |x| of a tile maps to 448.  The
+ * floor 1e-4 keeps an all-zero tile finite.  x is bf16.
+ */
+
+/* e4m3 code of a float: round to nearest, ties to even, from the bit layout
+ * above.  |x| >= 448 (infinities included) saturates to +-448; NaN gives 0x7F.
+ * Binade [2^E, 2^(E+1)) with E >= -6 is spaced 2^(E-3); below 2^-6 the
+ * subnormal spacing 2^-9 applies.                                           */
+uint8_t dgo_e4m3_encode(float x) {
+    if (isnan(x)) return 0x7F;
+    const uint8_t sign = signbit(x) ? 0x80 : 0x00;
+    const double a = fabs((double)x);
+    if (a >= 448.0) return sign | 0x7E;
+    if (a == 0.0) return sign;
+    int E;
+    frexp(a, &E); /* a = f * 2^E, f in [0.5, 1): a in [2^(E-1), 2^E) */
+    E -= 1;
+    if (E < -6) E = -6;
+    const double ulp = ldexp(1.0, E - 3);
+    const double q = a / ulp; /* exact: division by a power of two */
+    double f = floor(q);
+    const double rem = q - f;
+    if (rem > 0.5 || (rem == 0.5 && fmod(f, 2.0) == 1.0)) f += 1.0;
+    const double v = f * ulp; /* <= 448: every a < 448 rounds to at most 448 */
+    if (v < ldexp(1.0, -6)) return sign | (uint8_t)(v / ldexp(1.0, -9)); /* subnormal */
+    int E2;
+    frexp(v, &E2);
+    E2 -= 1; /* v may have rounded up into the next binade */
+    const int mant = (int)((v / ldexp(1.0, E2) - 1.0) * 8.0);
+    return sign | (uint8_t)(((E2 + 7) << 3) | mant);
+}
+
+static float bf16_bits_to_float(uint16_t h) {
+    uint32_t u = (uint32_t)h << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return f;
+}
+
+/* One tile: rows [r0, r1) x columns [c0, c0+128) of a row-major bf16 [.][K]. */
+static void cast_tile(const uint16_t* X, int64_t K, int r0, int r1, int c0, uint8_t* Q, float* s_out) {
+    float amax = 0.0f;
+    for (int r = r0; r < r1; ++r)
+        for (int k = c0; k < c0 + 128; ++k) amax = fmaxf(amax, fabsf(bf16_bits_to_float(X[r * K + k])));
+    amax = fmaxf(amax, 1e-4f);
+    const float s = amax / 448.0f;
+    const float rcp = 448.0f / amax;
+    *s_out = s;
+    for (int r = r0; r < r1; ++r)
+        for (int k = c0; k < c0 + 128; ++k) {
+            const float y = bf16_bits_to_float(X[r * K + k]) * rcp;
+            Q[r * K + k] = dgo_e4m3_encode(y);
+        }
+}
+
+/* Activations: X bf16 [M][K] -> Q e4m3 [M][K], sa[kb*sa_stride + m] (the
+ * GEMM's transposed layout).  K % 128 == 0, sa_stride >= M.                */
+int dgo_cast_1x128(const uint16_t* X, int M, int K, uint8_t* Q, float* sa, int64_t sa_stride) {
+    if (M < 0 || K <= 0 || K % 128 != 0 || sa_stride < M || !X || !Q || !sa) return DGO_BAD_ARG;
+    const int nkb = K / 128;
+#pragma omp parallel for schedule(static)
+    for (int m = 0; m < M; ++m)
+        for (int kb = 0; kb < nkb; ++kb) cast_tile(X, K, m, m + 1, kb * 128, Q, sa + (int64_t)kb * sa_stride + m);
+    return DGO_OK;
+}
+
+/* Weights: W bf16 [N][K] -> Q e4m3 [N][K], sb[nb*nkb + kb] with one scale per
+ * 128x128 block (the last row block may be shorter).  K % 128 == 0.        */
+int dgo_cast_128x128(const uint16_t* W, int N, int K, uint8_t* Q, float* sb) {
+    if (N < 0 || K <= 0 || K % 128 != 0 || !W || !Q || !sb) return DGO_BAD_ARG;
+    const int nkb = K / 128, nbn = (N + 127) / 128;
+#pragma omp parallel for schedule(static)
+    for (int nb = 0; nb < nbn; ++nb) {
+        const int r1 = (nb + 1) * 128 < N ? (nb + 1) * 128 : N;
+        for (int kb = 0; kb < nkb; ++kb) cast_tile(W, K, nb * 128, r1, kb * 128, Q, sb + (int64_t)nb * nkb + kb);
+    }
+    return DGO_OK;
+}
+
+void dgo_e4m3_encode_array(const float* x, uint8_t* out, int64_t n) {
+    for (int64_t i = 0; i < n; ++i) out[i] = dgo_e4m3_encode(x[i]);
+}

@@ -26,6 +26,14 @@ MUTANTS = {
     "contiguous_ignores_group": ("B + (int64_t)g * N * K, sb + (int64_t)g * nbn * nkb, N, K,\n                 D + m * N",
                                  "B, sb, N, K,\n                 D + m * N"),
     "masked_off_by_one": ("if (m >= masked_m[g]) continue;", "if (m > masked_m[g]) continue;"),
+    "cast_ties_away": ("if (rem > 0.5 || (rem == 0.5 && fmod(f, 2.0) == 1.0)) f += 1.0;", "if (rem >= 0.5) f += 1.0;"),
+    "cast_sign_lost": ("const uint8_t sign = signbit(x) ? 0x80 : 0x00;", "const uint8_t sign = 0x00;"),
+    "cast_no_floor": ("amax = fmaxf(amax, 1e-4f);", "amax = fmaxf(amax, 0.0f);"),
+    "cast_no_saturation": ("if (a >= 448.0) return sign | 0x7E;", "if (a >= 1e30) return sign | 0x7E;"),
+    "cast_half_tile_amax": ("for (int k = c0; k < c0 + 128; ++k) amax = fmaxf",
+                            "for (int k = c0; k < c0 + 64; ++k) amax = fmaxf"),
+    "cast_sa_not_transposed": ("cast_tile(X, K, m, m + 1, kb * 128, Q, sa + (int64_t)kb * sa_stride + m);",
+                               "cast_tile(X, K, m, m + 1, kb * 128, Q, sa + (int64_t)m * nkb + kb);"),
 }
 
 

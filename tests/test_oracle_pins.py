@@ -372,3 +372,130 @@ def test_case_bytes_adds_only_scales_and_indices():
     c = wl.dense_case(64, 256, 256, seed=0)
     base = 64 * 256 + 256 * 256 + 2 * 64 * 256
     assert base < c.bytes() <= base * 1.02
+
+
+# ------------------------------------------------------------- FP8 cast --
+# The cast ahead of the GEMM (activations per 1x128 tile, weights per 128x128
+# block): amax = max(max|x|, 1e-4), s = amax/448, q = e4m3_rne_satfinite(x*(448/amax)).
+
+def _finite_codes():
+    return [c for c in range(256) if c not in (0x7F, 0xFF)]
+
+
+def test_e4m3_encode_inverts_decode_on_every_finite_code():
+    codes = np.array(_finite_codes(), dtype=np.uint8)
+    vals = dequant_torch(codes).astype(np.float32)
+    assert np.array_equal(oracle.e4m3_encode(vals), codes)
+
+
+def test_e4m3_encode_matches_torch_cast_including_ties():
+    pos = np.array(sorted(set(np.abs(dequant_torch(np.arange(0, 0x7F, dtype=np.uint8))))))
+    mids = (pos[:-1] + pos[1:]) / 2  # exact ties, representable in float32
+    rng = np.random.default_rng(7)
+    rand = rng.uniform(-448, 448, 20000)
+    small = rng.uniform(-2 ** -5, 2 ** -5, 5000)  # subnormal range
+    x = np.concatenate([mids, -mids, rand, small, pos, -pos]).astype(np.float32)
+    ref = torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(oracle.e4m3_encode(x), ref)
+
+
+def test_e4m3_encode_saturates_and_keeps_nan():
+    x = np.array([448.0, 449.0, 464.0, 1e6, np.inf, -np.inf, -1e30, np.nan], dtype=np.float32)
+    assert oracle.e4m3_encode(x).tolist() == [0x7E, 0x7E, 0x7E, 0x7E, 0x7E, 0xFE, 0xFE, 0x7F]
+
+
+def _bf16_bits(x: np.ndarray) -> np.ndarray:
+    return torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32)).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+
+
+def _bf16_vals(bits: np.ndarray) -> np.ndarray:
+    return (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def _cast_inputs(M, K, seed):
+    rng = np.random.default_rng(seed)
+    x = rng.standard_normal((M, K)) * np.exp(rng.uniform(-6, 6, (M, 1)))
+    x[0, :128] = 0.0                    # an all-zero tile
+    x[M - 1, 128:256] *= 1e-7           # a tile below the 1e-4 floor
+    x[M // 2, 5] = 3e4                  # an outlier dominating one tile
+    return _bf16_bits(x)
+
+
+def _check_cast(X, Q, s_tile, tiles):
+    """tiles: list of (row slice, col slice) with scale s_tile[i]."""
+    xv = _bf16_vals(X)
+    qv = dequant_torch(Q)
+    for (rs, cs), s in zip(tiles, s_tile):
+        x, q = xv[rs, cs], qv[rs, cs]
+        amax = max(np.abs(x).max(), 1e-4)
+        assert s == np.float32(np.float32(amax) / np.float32(448.0))
+        if np.abs(x).max() >= 1e-4:
+            assert np.abs(q).max() == 448.0          # the largest |x| maps to 448
+        err = np.abs(s * q - x)
+        assert np.all(err <= 2.0 ** -4 * np.abs(x) * (1 + 2.0 ** -20) + s * 2.0 ** -10 + np.abs(x) * 2.0 ** -20)
+
+
+def test_cast_1x128_tiles_scales_and_layout():
+    M, K, stride = 37, 384, 40
+    X = _cast_inputs(M, K, 1)
+    Q, sa = oracle.cast_1x128(X, M, K, stride)
+    tiles = [(slice(m, m + 1), slice(kb * 128, kb * 128 + 128)) for m in range(M) for kb in range(K // 128)]
+    scales = [sa[kb * stride + m] for m in range(M) for kb in range(K // 128)]
+    _check_cast(X, Q, scales, tiles)
+    pad = np.concatenate([sa[kb * stride + M:(kb + 1) * stride] for kb in range(K // 128)])
+    assert np.all(pad == 0)                           # padding of sa_stride untouched
+
+
+def test_cast_128x128_tiles_and_ragged_rows():
+    N, K = 200, 256
+    W = _cast_inputs(N, K, 2)
+    Q, sb = oracle.cast_128x128(W, N, K)
+    assert sb.shape == (2, 2)
+    tiles = [(slice(nb * 128, min(N, nb * 128 + 128)), slice(kb * 128, kb * 128 + 128))
+             for nb in range(2) for kb in range(2)]
+    _check_cast(W, Q, sb.reshape(-1), tiles)
+
+
+@pytest.mark.parametrize("k", [-3, 5])
+def test_cast_is_invariant_under_power_of_two_scaling(k):
+    M, K = 9, 256
+    X = _cast_inputs(M, K, 3)
+    X2 = _bf16_bits(_bf16_vals(X) * 2.0 ** k)
+    assert np.array_equal(_bf16_vals(X2), _bf16_vals(X) * 2.0 ** k)  # exact in bf16
+    Q, sa = oracle.cast_1x128(X, M, K, M)
+    Q2, sa2 = oracle.cast_1x128(X2, M, K, M)
+    keep = np.repeat((np.abs(_bf16_vals(X)).reshape(M, -1, 128).max(axis=2) * 2.0 ** min(k, 0) >= 1e-4)
+                     .T.reshape(-1), 1)
+    assert np.array_equal(sa2[keep], sa[keep] * np.float32(2.0 ** k))
+    rows = np.repeat(keep.reshape(K // 128, M).T, 128, axis=1)
+    assert np.array_equal(Q2[rows], Q[rows])
+
+
+def test_cast_sign_symmetry_and_tile_independence():
+    M, K = 6, 384
+    X = _cast_inputs(M, K, 4)
+    Q, sa = oracle.cast_1x128(X, M, K, M)
+    Qn, san = oracle.cast_1x128(X ^ np.uint16(0x8000), M, K, M)
+    assert np.array_equal(san, sa)
+    assert np.array_equal(Qn[Q != 0], Q[Q != 0] ^ np.uint8(0x80))
+    X3 = X.copy()
+    X3[2, 130] = _bf16_bits(np.array([_bf16_vals(X[2:3, 130])[0] * 64 + 1.0]))[0]
+    Q3, sa3 = oracle.cast_1x128(X3, M, K, M)
+    changed = np.argwhere(Q3 != Q)
+    assert len(changed) and np.all(changed[:, 0] == 2) and np.all((changed[:, 1] >= 128) & (changed[:, 1] < 256))
+    assert [i for i in range(sa.size) if sa3[i] != sa[i]] == [1 * M + 2]
+
+
+def test_cast_then_gemm_tracks_the_bf16_product():
+    # The cast's sa / sb layouts must be the ones the GEMM reads: the GEMM of
+    # the cast operands stays close to the FP64 product of the bf16 inputs.
+    rng = np.random.default_rng(5)
+    M, N, K = 24, 260, 384
+    Xb = _bf16_bits(rng.standard_normal((M, K)) * np.exp(rng.uniform(-3, 3, (M, 1))))
+    Wb = _bf16_bits(0.02 * rng.standard_normal((N, K)) * np.exp(rng.uniform(-2, 2, (1, K))))
+    A, sa = oracle.cast_1x128(Xb, M, K, M)
+    B, sb = oracle.cast_128x128(Wb, N, K)
+    _, D64, _ = oracle.gemm_nt(A, sa, M, B, sb, M, N, K)
+    ref = _bf16_vals(Xb) @ _bf16_vals(Wb).T
+    rel = np.linalg.norm(D64 - ref) / np.linalg.norm(ref)
+    assert rel < 0.05
