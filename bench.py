@@ -294,6 +294,56 @@ class RotatingGraph:
         return self.ev[0].elapsed_time(self.ev[1]) * 1e-3 / self.launches
 
 
+# FP8 cast workloads: (kind, rows, K); "1x128" = activations, "128x128" = weights.
+CAST_SHAPES = [("1x128", 4096, 7168), ("1x128", 32768, 7168), ("1x128", 128, 7168), ("1x128", 64, 7168),
+               ("128x128", 7168, 16384), ("128x128", 4096, 7168)]
+
+
+def time_casts(dg, launches: int, warmup: int, stream) -> list:
+    """Each cast shape as a CUDA graph of `launches` calls over input copies
+    larger than L2 (like the GEMMs); one untimed replay first."""
+    out = []
+    for kind, R, K in CAST_SHAPES:
+        in_bytes = R * K * 2
+        copies = min(64, max(2, -(-ROTATE_FACTOR * L2_BYTES // (in_bytes + R * K))))
+        g = torch.Generator(device="cuda").manual_seed(R + K)
+        X0 = torch.randn(R, K, generator=g, device="cuda").to(torch.bfloat16)
+        bufs = []
+        for _ in range(copies):
+            nsc = (K // 128) * R if kind == "1x128" else -(-R // 128) * (K // 128)
+            bufs.append((X0.clone(), torch.empty(R, K, dtype=torch.uint8, device="cuda"),
+                         torch.empty(nsc, dtype=torch.float32, device="cuda")))
+
+        def call(i):
+            X, Q, sc = bufs[i % copies]
+            if kind == "1x128":
+                dg.dg_to_fp8_1x128(Q, sc, R, X)
+            else:
+                dg.dg_to_fp8_128x128(Q, sc, X)
+
+        with torch.cuda.stream(stream):
+            for i in range(max(warmup, 1) * copies):
+                call(i)
+        stream.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream):
+            for i in range(launches):
+                call(i)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            graph.replay()
+            e0.record(stream)
+            graph.replay()
+            e1.record(stream)
+        torch.cuda.synchronize()
+        t = e0.elapsed_time(e1) * 1e-3 / launches
+        nbytes = R * K * 3 + 4 * R * (K // 128) if kind == "1x128" else R * K * 3 + 4 * (-(-R // 128)) * (K // 128)
+        out.append({"cast": kind, "rows": R, "K": K, "us": round(t * 1e6, 2), "gbs": round(nbytes / t / 1e9, 1),
+                    "algorithmic_bytes": nbytes, "input_copies": copies})
+        del graph, bufs
+    return out
+
+
 def oracle_rows_sample(c: wl.Case, nrows: int, salt: int = 0):
     """A deterministic spread of nrows distinct row indices of a case."""
     import numpy as np
@@ -445,6 +495,10 @@ def run_ours(args, rank, world, local):
             "frac_roof_measured": round(roof_time_s(p.flops, p.bytes, p_fp8_sust, peaks["hbm_gbs"]) / tm, 3),
             "kernel": p.kernel, "us_flushed": round(statistics.median(tf) * 1e6, 2)})
 
+    casts = [] if args.no_grouped else time_casts(dg, max(3, min(args.steps, 20)), args.warmup, cap_stream)
+    for c in casts:
+        c["frac_hbm_measured"] = round(c["gbs"] / peaks["hbm_gbs"], 3)
+
     e2e = None
     if not args.no_e2e:
         # end to end: pinned host inputs -> device, GEMM, D -> pinned host
@@ -498,6 +552,7 @@ def run_ours(args, rank, world, local):
                    "wall_ms_per_step": round(t_wall / args.steps * 1e3, 3)},
         "per_shape": per_shape,
         "grouped": grouped_out,
+        "cast": casts,
         "roofline": roof,
         "cpu_baseline": cpu,
         "e2e": e2e,

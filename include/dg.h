@@ -117,6 +117,38 @@ DG_API dg_status dg_fp8_gemm_nt_noalloc(uint16_t* D, const uint8_t* A, const flo
                                         const uint8_t* B, const float* sb, int M, int N, int K, void* stream);
 
 /*
+ * FP8 cast of activations (the GEMM's A and sa).  The pages leave the cast to
+ * the caller ("接口": e4m3 inputs, transposed TMA-aligned LHS scales) and name
+ * a helper to_fp8 returning the FP8 tensor with its scale factors (the
+ * later-version article on DeepGEMM, section 4.1); one scale per 1x128 tile
+ * ("Deepseek DeepGEMM 技术原理的深入分析", section "技术背景与核心原理").
+ * Per tile, in IEEE single precision:
+ *   amax = max(max |x|, 1e-4),  s = amax / 448,
+ *   q = e4m3 of x * (448 / amax), round to nearest even, saturating to +-448
+ *   (NaN in, NaN out).
+ *   Q          uint8 e4m3 [M][K] (written)
+ *   sa         float32, sa[kb*sa_stride + m], kb < K/128 (written; the rest of
+ *              each sa_stride run is left untouched)
+ *   X          uint16 bf16 [M][K] (read)
+ * K % 128 == 0, sa_stride >= M (a multiple of 4 for the GEMM's TMA), X and Q
+ * 16-byte aligned.  M == 0 is valid and launches nothing.
+ */
+DG_API dg_status dg_to_fp8_1x128(uint8_t* Q, float* sa, int sa_stride, const uint16_t* X, int M, int K,
+                                 void* stream);
+
+/*
+ * FP8 cast of weights (the GEMM's B and sb), one scale per 128x128 block, the
+ * same steps as dg_to_fp8_1x128 over each block (the last row block may be
+ * shorter than 128).
+ *   Q          uint8 e4m3 [N][K] (written)
+ *   sb         float32 [ceil(N/128)][K/128], row-major (written)
+ *   W          uint16 bf16 [N][K] (read)
+ * K % 128 == 0, W and Q 16-byte aligned.  N == 0 is valid and launches nothing.
+ * For a grouped [G][N][K] weight, call once per group with the group's slices.
+ */
+DG_API dg_status dg_to_fp8_128x128(uint8_t* Q, float* sb, const uint16_t* W, int N, int K, void* stream);
+
+/*
  * Grouped GEMM, contiguous layout (section "分组 GEMM（连续布局）"): the rows of
  * all groups are concatenated along M and share N and K.  m_indices[m] (int32,
  * device) is the group of row m; -1 marks a padding row, whose D row is left

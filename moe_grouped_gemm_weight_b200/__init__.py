@@ -58,6 +58,10 @@ def lib() -> ctypes.CDLL:
             L.dg_fp8_gemm_nt.argtypes = [P, P, P, I, P, P, I, I, I, P]
             L.dg_fp8_gemm_nt_noalloc.restype = I
             L.dg_fp8_gemm_nt_noalloc.argtypes = [P, P, P, I, P, P, I, I, I, P]
+            L.dg_to_fp8_1x128.restype = I
+            L.dg_to_fp8_1x128.argtypes = [P, P, I, P, I, I, P]
+            L.dg_to_fp8_128x128.restype = I
+            L.dg_to_fp8_128x128.argtypes = [P, P, P, I, I, P]
             L.dg_grouped_contiguous_nt.restype = I
             L.dg_grouped_contiguous_nt.argtypes = [P, P, P, I, P, P, P, I, I, I, I, P]
             L.dg_grouped_masked_nt.restype = I
@@ -119,6 +123,19 @@ def dg_fp8_gemm_nt_noalloc(D, A, sa, sa_stride: int, B, sb, stream=None) -> None
     _check("dg_fp8_gemm_nt_noalloc",
            lib().dg_fp8_gemm_nt_noalloc(_ptr(D), _ptr(A), _ptr(sa), int(sa_stride), _ptr(B), _ptr(sb),
                                         M, N, K, _stream(stream)))
+
+
+def dg_to_fp8_1x128(Q, sa, sa_stride: int, X, stream=None) -> None:
+    """Activation cast: bf16 X [M,K] -> e4m3 Q [M,K] (uint8) and sa[kb*sa_stride + m]."""
+    M, K = X.shape[-2], X.shape[-1]
+    _check("dg_to_fp8_1x128", lib().dg_to_fp8_1x128(_ptr(Q), _ptr(sa), int(sa_stride), _ptr(X), M, K,
+                                                    _stream(stream)))
+
+
+def dg_to_fp8_128x128(Q, sb, W, stream=None) -> None:
+    """Weight cast: bf16 W [N,K] -> e4m3 Q [N,K] (uint8) and sb [ceil(N/128), K/128]."""
+    N, K = W.shape[-2], W.shape[-1]
+    _check("dg_to_fp8_128x128", lib().dg_to_fp8_128x128(_ptr(Q), _ptr(sb), _ptr(W), N, K, _stream(stream)))
 
 
 def dg_grouped_contiguous_nt(D, A, sa, sa_stride: int, B, sb, m_indices, stream=None) -> None:

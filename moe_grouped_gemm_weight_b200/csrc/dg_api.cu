@@ -20,6 +20,7 @@
 #include "dg_kernel.cuh"
 #include "dg_kernel_small.cuh"
 #include "dg_kernel_pair.cuh"
+#include "dg_cast.cuh"
 
 namespace dg {
 // One CTA waits (bounded) on a barrier that no one arrives at.
@@ -815,6 +816,56 @@ dg_status dg_grouped_masked_nt(uint16_t* D, const uint8_t* A, const float* sa, i
     p.b_stream = M_max <= dg::kBM;
     if (pl.cta_pair) return launch_pair<dg::kMasked>(p, ta, tb, td, pl, static_cast<cudaStream_t>(stream));
     return dispatch<dg::kMasked>(pl, p, ta, tb, td, static_cast<cudaStream_t>(stream));
+}
+
+dg_status dg_to_fp8_1x128(uint8_t* Q, float* sa, int sa_stride, const uint16_t* X, int M, int K, void* stream) {
+    if (M < 0 || K <= 0) return fail(DG_ERR_INVALID_ARG, "bad sizes M=%d K=%d", M, K);
+    if (K % dg::kBK != 0) return fail(DG_ERR_UNSUPPORTED, "K=%d must be a multiple of 128", K);
+    if (!Q || !sa || !X) return fail(DG_ERR_INVALID_ARG, "null pointer");
+    if (!aligned16(Q) || !aligned16(X) || (reinterpret_cast<uintptr_t>(sa) & 3u))
+        return fail(DG_ERR_MISALIGNED, "X and Q must be 16-byte aligned, sa 4-byte aligned");
+    if (sa_stride < M) return fail(DG_ERR_INVALID_ARG, "sa_stride=%d must be >= M=%d", sa_stride, M);
+    if (M == 0) return ok();
+    const int sms = effective_sms();
+    if (sms <= 0) return fail(DG_ERR_CUDA, "no CUDA device");
+    dg::CastParams p{Q, sa, X, M, K, K / dg::kBK, sa_stride};
+    const int64_t items = static_cast<int64_t>(cdiv(M, dg::kCastRowsPerCta)) * cdiv(K / dg::kBK, dg::kCastBlocks);
+    const int64_t cap = static_cast<int64_t>(sms) * 8;  // 8 CTAs of 256 threads per SM
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(items < cap ? items : cap), 1, 1);
+    cfg.blockDim = dim3(dg::kCastThreads, 1, 1);
+    cfg.stream = static_cast<cudaStream_t>(stream);
+    cudaLaunchAttribute attr[1];
+    set_pdl(attr[0]);
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, dg::cast_1x128_kernel, p);
+    if (e == cudaSuccess) e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(DG_ERR_CUDA, "kernel launch failed: %s", cudaGetErrorString(e));
+    return ok();
+}
+
+dg_status dg_to_fp8_128x128(uint8_t* Q, float* sb, const uint16_t* W, int N, int K, void* stream) {
+    if (N < 0 || K <= 0) return fail(DG_ERR_INVALID_ARG, "bad sizes N=%d K=%d", N, K);
+    if (K % dg::kBK != 0) return fail(DG_ERR_UNSUPPORTED, "K=%d must be a multiple of 128", K);
+    if (!Q || !sb || !W) return fail(DG_ERR_INVALID_ARG, "null pointer");
+    if (!aligned16(Q) || !aligned16(W) || (reinterpret_cast<uintptr_t>(sb) & 3u))
+        return fail(DG_ERR_MISALIGNED, "W and Q must be 16-byte aligned, sb 4-byte aligned");
+    if (N == 0) return ok();
+    if (cdiv(N, 128) > 65535) return fail(DG_ERR_UNSUPPORTED, "N=%d too large", N);
+    dg::CastParams p{Q, sb, W, N, K, K / dg::kBK, 0};
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(K / dg::kBK), static_cast<unsigned>(cdiv(N, 128)), 1);
+    cfg.blockDim = dim3(dg::kCastThreads, 1, 1);
+    cfg.stream = static_cast<cudaStream_t>(stream);
+    cudaLaunchAttribute attr[1];
+    set_pdl(attr[0]);
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, dg::cast_128x128_kernel, p);
+    if (e == cudaSuccess) e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(DG_ERR_CUDA, "kernel launch failed: %s", cudaGetErrorString(e));
+    return ok();
 }
 
 void dg_set_num_sms(int n) { g_num_sms_cap.store(n > 0 ? n : 0); }

@@ -142,6 +142,23 @@ def test_gemm_calls_reject_bad_arguments_without_touching_the_gpu():
         dg.dg_get_num_sms() > 0
 
 
+def test_cast_calls_reject_bad_arguments_without_touching_the_gpu():
+    L = dg.lib()
+    fake = 1 << 20  # never dereferenced: every call below fails validation first
+    st = L.dg_to_fp8_1x128(fake, fake, 64, fake, 64, 100, 0)
+    assert st == dg.DG_ERR_UNSUPPORTED and b"K=100" in L.dg_last_error_message()
+    assert L.dg_to_fp8_1x128(0, fake, 64, fake, 64, 128, 0) == dg.DG_ERR_INVALID_ARG
+    assert L.dg_to_fp8_1x128(fake, fake, 64, fake + 8, 64, 128, 0) == dg.DG_ERR_MISALIGNED
+    assert L.dg_to_fp8_1x128(fake, fake + 2, 64, fake, 64, 128, 0) == dg.DG_ERR_MISALIGNED
+    assert L.dg_to_fp8_1x128(fake, fake, 63, fake, 64, 128, 0) == dg.DG_ERR_INVALID_ARG
+    assert L.dg_to_fp8_1x128(fake, fake, 64, fake, -1, 128, 0) == dg.DG_ERR_INVALID_ARG
+    assert L.dg_to_fp8_1x128(fake, fake, 0, fake, 0, 128, 0) == dg.DG_OK  # empty: nothing launched
+    assert L.dg_to_fp8_128x128(fake, fake, fake, 64, 130, 0) == dg.DG_ERR_UNSUPPORTED
+    assert L.dg_to_fp8_128x128(fake, 0, fake, 64, 128, 0) == dg.DG_ERR_INVALID_ARG
+    assert L.dg_to_fp8_128x128(fake + 4, fake, fake, 64, 128, 0) == dg.DG_ERR_MISALIGNED
+    assert L.dg_to_fp8_128x128(fake, fake, fake, 0, 128, 0) == dg.DG_OK
+
+
 def test_empty_problem_is_a_no_op():
     L = dg.lib()
     fake = 1 << 20
