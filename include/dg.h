@@ -180,6 +180,20 @@ DG_API dg_status dg_grouped_masked_nt(uint16_t* D, const uint8_t* A, const float
 
 /* Utility functions (section "工具函数" (utility functions) of the same page). */
 
+/*
+ * Programmatic dependent launch (the later-version article on DeepGEMM,
+ * section 4.3, enables it with set_pdl(True)).  When on, every launch of this
+ * library may start its set-up while the previous kernel in the stream is
+ * finishing; the kernels wait for that kernel's results before touching global
+ * memory, so results never change.  Off by default (measured: it shortens some
+ * decode-sized launches and lengthens large cluster launches).
+ *   dg_set_pdl(1) on, dg_set_pdl(0) off, dg_set_pdl(-1) back to the default,
+ *   which reads the environment variable DG_PDL=1 at every launch.
+ * Process-global, like dg_set_num_sms.  dg_get_pdl returns the current state.
+ */
+DG_API void dg_set_pdl(int enable);
+DG_API int dg_get_pdl(void);
+
 /* Cap the number of SMs the persistent kernels use (n <= 0: all SMs). */
 DG_API void dg_set_num_sms(int n);
 /* Current cap; the device's SM count when no cap is set (0 without a GPU). */

@@ -66,6 +66,10 @@ def lib() -> ctypes.CDLL:
             L.dg_grouped_contiguous_nt.argtypes = [P, P, P, I, P, P, P, I, I, I, I, P]
             L.dg_grouped_masked_nt.restype = I
             L.dg_grouped_masked_nt.argtypes = [P, P, P, I, P, P, P, I, I, I, I, I, P]
+            L.dg_set_pdl.restype = None
+            L.dg_set_pdl.argtypes = [I]
+            L.dg_get_pdl.restype = I
+            L.dg_get_pdl.argtypes = []
             L.dg_set_num_sms.restype = None
             L.dg_set_num_sms.argtypes = [I]
             L.dg_get_num_sms.restype = I
@@ -154,6 +158,15 @@ def dg_grouped_masked_nt(D, A, sa, sa_stride: int, B, sb, masked_m, expected_m: 
     _check("dg_grouped_masked_nt",
            lib().dg_grouped_masked_nt(_ptr(D), _ptr(A), _ptr(sa), int(sa_stride), _ptr(B), _ptr(sb),
                                       _ptr(masked_m), G, Mmax, N, K, int(expected_m), _stream(stream)))
+
+
+def dg_set_pdl(enable) -> None:
+    """Programmatic dependent launch on (True), off (False) or default (None: DG_PDL=1)."""
+    lib().dg_set_pdl(-1 if enable is None else int(bool(enable)))
+
+
+def dg_get_pdl() -> bool:
+    return bool(lib().dg_get_pdl())
 
 
 def dg_set_num_sms(n: int) -> None:

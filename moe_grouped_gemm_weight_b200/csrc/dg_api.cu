@@ -357,7 +357,11 @@ dg_status plan(int mode, int rows, int N, int K, int G, int num_sms, dg_plan* ou
 // 64x32768x512 by about a quarter) but lengthens cluster launches with large
 // grids (64x7168x16384 by up to a third), whose CTAs are then placed into
 // slots as the previous grid frees them instead of spread over an idle GPU.
+std::atomic<int> g_pdl{-1};  // -1: from DG_PDL, else 0 / 1 from dg_set_pdl
+
 bool pdl_enabled() {
+    const int set = g_pdl.load();
+    if (set >= 0) return set != 0;
     const char* v = std::getenv("DG_PDL");
     return v && v[0] == '1';
 }
@@ -867,6 +871,10 @@ dg_status dg_to_fp8_128x128(uint8_t* Q, float* sb, const uint16_t* W, int N, int
     if (e != cudaSuccess) return fail(DG_ERR_CUDA, "kernel launch failed: %s", cudaGetErrorString(e));
     return ok();
 }
+
+void dg_set_pdl(int enable) { g_pdl.store(enable < 0 ? -1 : (enable ? 1 : 0)); }
+
+int dg_get_pdl(void) { return pdl_enabled() ? 1 : 0; }
 
 void dg_set_num_sms(int n) { g_num_sms_cap.store(n > 0 ? n : 0); }
 

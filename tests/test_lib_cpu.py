@@ -172,3 +172,19 @@ def test_binding_fails_loudly_when_library_missing(tmp_path, monkeypatch):
     monkeypatch.setattr(mod, "LIB_PATH", str(tmp_path / "missing.so"))
     with pytest.raises(RuntimeError, match="missing"):
         mod.dg_get_num_sms()
+
+
+def test_pdl_switch_defaults_to_the_environment(monkeypatch):
+    try:
+        dg.dg_set_pdl(None)
+        monkeypatch.setenv("DG_PDL", "1")
+        assert dg.dg_get_pdl() is True
+        monkeypatch.setenv("DG_PDL", "0")
+        assert dg.dg_get_pdl() is False
+        dg.dg_set_pdl(True)
+        assert dg.dg_get_pdl() is True
+        dg.dg_set_pdl(False)
+        monkeypatch.setenv("DG_PDL", "1")
+        assert dg.dg_get_pdl() is False
+    finally:
+        dg.dg_set_pdl(None)
