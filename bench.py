@@ -294,6 +294,51 @@ class RotatingGraph:
         return self.ev[0].elapsed_time(self.ev[1]) * 1e-3 / self.launches
 
 
+class Ue8m0Problem(Problem):
+    """A dense problem with power-of-two scales, run through a chosen entry
+    point: "promote" (dg_fp8_gemm_nt), "ue8m0" (dg_fp8_gemm_nt_ue8m0, routed)
+    or "block_scaled" (the same call with DG_FORCE_BLOCK_SCALED=1)."""
+
+    def __init__(self, case, dg, path):
+        super().__init__(case, dg)
+        self.path = path
+
+    def run(self, case=None, D=None):
+        c = case or self.case
+        D = self.D if D is None else D
+        if self.path == "promote":
+            self.dg.dg_fp8_gemm_nt(D, c.A, c.sa, c.sa_stride, c.B, c.sb)
+        else:
+            os.environ["DG_FORCE_BLOCK_SCALED"] = "1" if self.path == "block_scaled" else "0"
+            try:
+                self.dg.dg_fp8_gemm_nt_ue8m0(D, c.A, c.sa, c.sa_stride, c.B, c.sb)
+            finally:
+                os.environ.pop("DG_FORCE_BLOCK_SCALED", None)
+
+
+UE8M0_SHAPES = [(4096, 32768, 512), (4096, 24576, 1536), (4096, 7168, 2048), (4096, 7168, 16384)]
+
+
+def time_ue8m0(dg, launches: int, warmup: int, stream) -> list:
+    """Power-of-two scales (the stress generator): each shape through the three
+    paths, each as a CUDA graph over input copies larger than L2."""
+    out = []
+    for (m, n, k) in UE8M0_SHAPES:
+        case = wl.dense_case(m, n, k, seed=0, stress=True, device="cuda")
+        row = {"M": m, "N": n, "K": k}
+        for path in ("promote", "ue8m0", "block_scaled"):
+            pr = Ue8m0Problem(case, dg, path)
+            gr = RotatingGraph(pr, launches, warmup, stream)
+            gr.replay()
+            torch.cuda.synchronize()
+            t = gr.seconds_per_launch()
+            row[f"us_{path}"] = round(t * 1e6, 2)
+            row[f"tflops_{path}"] = round(pr.flops / t / 1e12, 1)
+            del gr
+        out.append(row)
+    return out
+
+
 # FP8 cast workloads: (kind, rows, K); "1x128" = activations, "128x128" = weights.
 CAST_SHAPES = [("1x128", 4096, 7168), ("1x128", 32768, 7168), ("1x128", 128, 7168), ("1x128", 64, 7168),
                ("128x128", 7168, 16384), ("128x128", 4096, 7168)]
@@ -496,6 +541,7 @@ def run_ours(args, rank, world, local):
             "kernel": p.kernel, "us_flushed": round(statistics.median(tf) * 1e6, 2)})
 
     casts = [] if args.no_grouped else time_casts(dg, max(3, min(args.steps, 20)), args.warmup, cap_stream)
+    ue8m0 = [] if args.no_grouped else time_ue8m0(dg, max(3, min(args.steps, 10)), args.warmup, cap_stream)
     for c in casts:
         c["frac_hbm_measured"] = round(c["gbs"] / peaks["hbm_gbs"], 3)
 
@@ -553,6 +599,7 @@ def run_ours(args, rank, world, local):
         "per_shape": per_shape,
         "grouped": grouped_out,
         "cast": casts,
+        "ue8m0": ue8m0,
         "roofline": roof,
         "cpu_baseline": cpu,
         "e2e": e2e,

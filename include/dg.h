@@ -79,6 +79,8 @@ typedef enum dg_status {
 #define DG_DEVERR_TIMEOUT 1u        /* a bounded wait inside a kernel ran out  */
 #define DG_DEVERR_BAD_M_INDEX 2u    /* contiguous: m_indices value not in [-1,G) */
 #define DG_DEVERR_BAD_MASKED_M 4u   /* masked: masked_m value not in [0,M_max]  */
+#define DG_DEVERR_NOT_POW2 8u       /* ue8m0 call: a scale is not a positive     */
+                                    /* normal power of two                       */
 
 /*
  * Dense GEMM: D[M,N] = scaled A[M,K] . B[N,K]^T (section "常规密集型 GEMM（非分组）",
@@ -92,6 +94,26 @@ typedef enum dg_status {
  */
 DG_API dg_status dg_fp8_gemm_nt(uint16_t* D, const uint8_t* A, const float* sa, int sa_stride,
                          const uint8_t* B, const float* sb, int M, int N, int K, void* stream);
+
+/*
+ * Dense GEMM for power-of-two scales, scaled inside the tensor core.  Same
+ * arguments, layouts and result as dg_fp8_gemm_nt, but every sa and sb value
+ * must be a positive normal power of two (UE8M0-representable: its FP32
+ * exponent field is the UE8M0 code).  The later-version article on DeepGEMM
+ * (section 3.1) notes that SM100 takes UE8M0 scales; this call hands them to
+ * tcgen05.mma kind::mxf8f6f4.block_scale, which applies them to each K=32
+ * partial product before the FP32 accumulation, instead of promoting every
+ * 128-K block through registers.  The result is the method's sum up to FP32
+ * summation order (tolerance as for dg_fp8_gemm_nt).  A scale that is not a
+ * power of two sets DG_DEVERR_NOT_POW2 in the device error word and its tile's
+ * results are then wrong; the call does not check the scales on the host.
+ * The block-scaled kernel is used where it measured faster than the promotion
+ * kernel (K <= 2048 with at least two waves of 128 x 256 tiles); other shapes
+ * take the promotion kernel (the same result, no DG_DEVERR_NOT_POW2 check).
+ * DG_FORCE_BLOCK_SCALED=1 in the environment forces the block-scaled kernel.
+ */
+DG_API dg_status dg_fp8_gemm_nt_ue8m0(uint16_t* D, const uint8_t* A, const float* sa, int sa_stride,
+                                      const uint8_t* B, const float* sb, int M, int N, int K, void* stream);
 
 /*
  * Dense GEMM that allocates nothing.  The pages describe no such call; it

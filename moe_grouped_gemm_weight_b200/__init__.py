@@ -24,7 +24,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libdg.so")
 
 DG_OK, DG_ERR_INVALID_ARG, DG_ERR_UNSUPPORTED, DG_ERR_MISALIGNED, DG_ERR_CUDA = range(5)
-DG_DEVERR_TIMEOUT, DG_DEVERR_BAD_M_INDEX, DG_DEVERR_BAD_MASKED_M = 1, 2, 4
+DG_DEVERR_TIMEOUT, DG_DEVERR_BAD_M_INDEX, DG_DEVERR_BAD_MASKED_M, DG_DEVERR_NOT_POW2 = 1, 2, 4, 8
 
 _lock = threading.Lock()
 _lib = None
@@ -56,6 +56,8 @@ def lib() -> ctypes.CDLL:
             P, I = ctypes.c_void_p, ctypes.c_int
             L.dg_fp8_gemm_nt.restype = I
             L.dg_fp8_gemm_nt.argtypes = [P, P, P, I, P, P, I, I, I, P]
+            L.dg_fp8_gemm_nt_ue8m0.restype = I
+            L.dg_fp8_gemm_nt_ue8m0.argtypes = [P, P, P, I, P, P, I, I, I, P]
             L.dg_fp8_gemm_nt_noalloc.restype = I
             L.dg_fp8_gemm_nt_noalloc.argtypes = [P, P, P, I, P, P, I, I, I, P]
             L.dg_to_fp8_1x128.restype = I
@@ -116,6 +118,14 @@ def dg_fp8_gemm_nt(D, A, sa, sa_stride: int, B, sb, stream=None) -> None:
     N = B.shape[-2]
     _check("dg_fp8_gemm_nt", lib().dg_fp8_gemm_nt(_ptr(D), _ptr(A), _ptr(sa), int(sa_stride), _ptr(B), _ptr(sb),
                                                   M, N, K, _stream(stream)))
+
+
+def dg_fp8_gemm_nt_ue8m0(D, A, sa, sa_stride: int, B, sb, stream=None) -> None:
+    """dg_fp8_gemm_nt for power-of-two sa / sb, scaled inside the tensor core."""
+    M, K = A.shape[-2], A.shape[-1]
+    N = B.shape[-2]
+    _check("dg_fp8_gemm_nt_ue8m0", lib().dg_fp8_gemm_nt_ue8m0(_ptr(D), _ptr(A), _ptr(sa), int(sa_stride), _ptr(B),
+                                                            _ptr(sb), M, N, K, _stream(stream)))
 
 
 def dg_fp8_gemm_nt_noalloc(D, A, sa, sa_stride: int, B, sb, stream=None) -> None:

@@ -21,6 +21,7 @@
 #include "dg_kernel_small.cuh"
 #include "dg_kernel_pair.cuh"
 #include "dg_cast.cuh"
+#include "dg_kernel_ue8m0.cuh"
 
 namespace dg {
 // One CTA waits (bounded) on a barrier that no one arrives at.
@@ -766,6 +767,70 @@ dg_status dg_fp8_gemm_nt_noalloc(uint16_t* D, const uint8_t* A, const float* sa,
         p.ws_flags = flags;
     }
     return dispatch<dg::kDense>(pl, p, ta, tb, td, st);
+}
+
+dg_status dg_fp8_gemm_nt_ue8m0(uint16_t* D, const uint8_t* A, const float* sa, int sa_stride, const uint8_t* B,
+                               const float* sb, int M, int N, int K, void* stream) {
+    dg_status s = check_sizes(0, M, N, K, 1);
+    if (s != DG_OK) return s;
+    if ((s = common_checks(D, A, sa, sa_stride, B, sb, M)) != DG_OK) return s;
+    if (M == 0) return ok();
+    const int sms = effective_sms();
+    if (sms <= 0) return fail(DG_ERR_CUDA, "no CUDA device");
+    // The block-scaled kernel has no K-split tail and a fixed 128 x 256 tile.
+    // Measured against the promotion kernel on power-of-two scales (CUDA-graph
+    // replays on B200) it is faster when K <= 2048 and there are at least two
+    // waves of tiles (4096x32768x512 by 25 %, 4096x24576x1536 by 8 %,
+    // 4096x7168x2048 by 3 %) and slower otherwise (4096x7168x16384 by 20 %,
+    // where the promotion kernel splits the partial last wave).  Elsewhere the
+    // call takes the promotion kernel, which computes the same sum for any
+    // FP32 scales.  DG_FORCE_BLOCK_SCALED=1 always takes the block-scaled one.
+    {
+        const char* force = std::getenv("DG_FORCE_BLOCK_SCALED");
+        const int ue_tiles = cdiv(M, dg::kBM) * cdiv(N, dg::kUeBN);
+        const bool block_scaled = (force && force[0] == '1') || (K <= 2048 && ue_tiles >= 2 * sms);
+        if (!block_scaled) return dg_fp8_gemm_nt(D, A, sa, sa_stride, B, sb, M, N, K, stream);
+    }
+    dg_plan pl{};
+    pl.block_m = dg::kBM;
+    pl.block_n = dg::kUeBN;
+    pl.stages = dg::kUeStages;
+    pl.m_blocks = cdiv(M, dg::kBM);
+    pl.n_blocks = cdiv(N, dg::kUeBN);
+    pl.tiles = pl.m_blocks * pl.n_blocks;
+    pl.grid = pl.tiles < sms ? pl.tiles : sms;
+    pl.split_k = 1;
+    pl.tail_split = 1;
+    CUtensorMap ta, tb, td;
+    if ((s = make_operand_map(&ta, A, K, M, 1, dg::kBM, false)) != DG_OK) return s;
+    if ((s = make_operand_map(&tb, B, K, N, 1, dg::kUeBN, true)) != DG_OK) return s;
+    if ((s = make_output_map(&td, D, N, M, 1, false)) != DG_OK) return s;
+    dg::Params p = make_params(D, sa, sa_stride, sb, M, N, K, 1, pl);
+    p.b_stream = pl.m_blocks == 1;
+    constexpr int smem = dg::ue8m0_smem_bytes();
+    static_assert(smem <= 227 * 1024, "shared memory budget exceeded");
+    auto kern = dg::fp8_gemm_ue8m0_kernel;
+    static std::atomic<int> attr_set[kMaxDevices];
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev >= 0 && dev < kMaxDevices && !attr_set[dev].load()) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+            return fail(DG_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(cudaGetLastError()));
+        attr_set[dev].store(1);
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(pl.grid), 1, 1);
+    cfg.blockDim = dim3(dg::kUeThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = static_cast<cudaStream_t>(stream);
+    cudaLaunchAttribute attr[1];
+    set_pdl(attr[0]);
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kern, p, ta, tb, td);
+    if (e == cudaSuccess) e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(DG_ERR_CUDA, "kernel launch failed: %s", cudaGetErrorString(e));
+    return ok();
 }
 
 dg_status dg_grouped_contiguous_nt(uint16_t* D, const uint8_t* A, const float* sa, int sa_stride, const uint8_t* B,

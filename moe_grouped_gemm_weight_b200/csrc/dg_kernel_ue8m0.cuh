@@ -1,0 +1,366 @@
+// dg_kernel_ue8m0.cuh -- sm_100a dense GEMM for power-of-two scales, scaled
+// inside the tensor core.
+//
+// When every scale is a power of two (UE8M0-representable: the FP32 value is
+// 2^e, its exponent field is the UE8M0 code), the scaled sum of the method
+//   D[m,n] = sum_kb sa[m,kb] * sb[n/128,kb] * sum_{k in kb} A[m,k] * B[n,k]
+// is what tcgen05.mma kind::mxf8f6f4.block_scale computes when it is given
+// one scale per row of A and one per column of B for every 32-wide K step:
+// the product of the two scales multiplies the step's partial sum before it
+// enters the FP32 accumulator in TMEM.  The 1x128 / 128x128 scales are simply
+// repeated over the four K=32 steps of each 128-wide K block.  No promotion
+// through registers is needed, so the accumulator stays in TMEM for a whole
+// tile and the epilogue reads it once.
+//
+// The pages' Hopper design promotes on CUDA cores because Hopper's FP8
+// tensor-core accumulation is not FP32 ("Deepseek DeepGEMM 技术原理的深入分析",
+// section "技术背景与核心原理"); the later-version article on DeepGEMM
+// (section 3.1) notes that on SM100 the scales are UE8M0.  This kernel is the
+// SM100 path for such scales; the general FP32-scale kernels stay the default.
+//
+// Tiles 128 x 256, persistent CTAs of 384 threads:
+//   warp 0      TMA producer (A 128x128 and B 256x128 per K block, 4 stages)
+//   warp 1      TMEM owner; per four K blocks copies their scale factors from
+//               shared memory to TMEM (tcgen05.cp); per K block issues 4 MMAs
+//   warp 2      scale loader: sa (128 rows) and sb (2 blocks) per K block by
+//               cp.async into an 8-slot FP32 ring
+//   warp 3      scale converter: FP32 -> UE8M0 codes in the scale-factor
+//               layout, 8-slot ring; a scale that is not a positive normal
+//               power of two sets DG_DEVERR_NOT_POW2 (its code is still its
+//               exponent field, so the result is wrong for it)
+//   warps 4-11  epilogue: TMEM -> bf16 -> TMA store (two warpgroups of 128
+//               columns)
+// Scale-factor layout in shared memory (one 512-byte block per 128 rows or
+// columns): the 32-bit word for row r sits at byte (r % 32) * 16 + (r / 32) * 4.
+// tcgen05.cp .32x128b.warpx4 places it in TMEM column (r / 32) of lane r % 32,
+// repeated in every 32-lane quarter.  Each MMA picks one byte of the word
+// (sf_id); since a scale is constant over a 128-wide K block, byte j holds
+// the code of the j-th K block of a group of four, and the four MMAs of that K
+// block all use sf_id = j: one copy to TMEM serves four K blocks.
+#pragma once
+
+#include "dg_kernel.cuh"
+
+namespace dg {
+
+constexpr int kUeBN = 256;
+constexpr int kUeStages = 4;
+constexpr int kUeSfSlots = 8;
+constexpr int kUeSfaBytes = 512;                       // 128 rows of A
+constexpr int kUeSfbBytes = 1024;                      // 256 columns of B
+constexpr int kUeSfSlotBytes = kUeSfaBytes + kUeSfbBytes;
+constexpr int kUeSfColsPerSlot = 12;                   // TMEM: 4 (A) + 8 (B)
+constexpr int kUeSfGroup = 4;                          // K blocks per scale-factor slot (one byte each)
+constexpr int kUeRawSlots = 8;                         // FP32 scales as loaded
+constexpr int kUeRawFloats = kBM + 4;                  // sa of 128 rows + 2 sb (16-byte padded)
+constexpr int kUeAccCols = kUeBN;                      // one FP32 accumulator
+constexpr int kUeTmemCols = 512;
+constexpr int kUeEpiWarps = 8;
+constexpr int kUeThreads = 32 * (kFirstEpiWarp + kUeEpiWarps);
+constexpr int kUeTileBBytes = kUeBN * kBK;
+static_assert(kUeAccCols + kUeSfSlots * kUeSfColsPerSlot <= kUeTmemCols, "TMEM budget");
+
+constexpr int ue8m0_smem_bytes() {
+    return 1024 + kUeStages * (kTileABytes + kUeTileBBytes) + kUeEpiWarps * kStageOutBytes +
+           kUeSfSlots * kUeSfSlotBytes + kUeRawSlots * kUeRawFloats * 4 + 512;
+}
+
+// UE8M0 code of a positive normal power of two; anything else raises the
+// error bit (and keeps its exponent field).
+__device__ __forceinline__ uint32_t ue8m0_code(float v) {
+    const uint32_t bits = __float_as_uint(v);
+    const uint32_t e = (bits >> 23) & 0xFFu;
+    if ((bits & 0x807FFFFFu) != 0u || e == 0u || e == 0xFFu) atomicOr(&g_dg_error, 8u);
+    return e;
+}
+
+__global__ void __launch_bounds__(kUeThreads, 1)
+fp8_gemm_ue8m0_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtensorMap tmA,
+                      const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmD) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* sA = smem;
+    uint8_t* sB = sA + kUeStages * kTileABytes;
+    uint8_t* sOut = sB + kUeStages * kUeTileBBytes;
+    uint8_t* sSF = sOut + kUeEpiWarps * kStageOutBytes;  // 512-byte aligned
+    float* sRaw = reinterpret_cast<float*>(sSF + kUeSfSlots * kUeSfSlotBytes);
+    uint64_t* full = reinterpret_cast<uint64_t*>(sRaw + kUeRawSlots * kUeRawFloats);
+    uint64_t* empty = full + kUeStages;
+    uint64_t* sf_full = empty + kUeStages;
+    uint64_t* sf_empty = sf_full + kUeSfSlots;
+    uint64_t* raw_full = sf_empty + kUeSfSlots;
+    uint64_t* raw_empty = raw_full + kUeRawSlots;
+    uint64_t* acc_full = raw_empty + kUeRawSlots;
+    uint64_t* acc_empty = acc_full + 1;
+    uint64_t* done = acc_empty + 1;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kUeStages; ++s) {
+            mbar_init(full + s, 1);
+            mbar_init(empty + s, 1);
+        }
+        for (int s = 0; s < kUeSfSlots; ++s) {
+            mbar_init(sf_full + s, 1);
+            mbar_init(sf_empty + s, 1);
+        }
+        for (int s = 0; s < kUeRawSlots; ++s) {
+            mbar_init(raw_full + s, 32);
+            mbar_init(raw_empty + s, 1);
+        }
+        mbar_init(acc_full, 1);
+        mbar_init(acc_empty, kUeEpiWarps);
+        mbar_init(done, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0) {
+        prefetch_tmap(&tmA);
+        prefetch_tmap(&tmB);
+        prefetch_tmap(&tmD);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, kUeTmemCols);
+        tmem_relinquish();
+    }
+    griddep_wait();
+    griddep_launch_dependents();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    const int tiles = p.m_blocks * p.n_blocks;
+    const int nkb = p.nkb;
+
+    if (warp < kFirstEpiWarp) {
+        regs_dec<56>();
+        if (warp == 0) {
+            // ------------------------------------------------------ producer ----
+            const uint64_t pol_a = l2_policy_evict_last();
+            const uint64_t pol_b = p.b_stream ? l2_policy_evict_first() : l2_policy_evict_last();
+            int stage = 0, fills = 0;
+            uint32_t phase = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; ok && t < tiles; t += gridDim.x) {
+                int mb, nb;
+                raster_tile(t, p.m_blocks, p.n_blocks, p.raster, mb, nb);
+                for (int kb = 0; kb < nkb; ++kb) {
+                    if (!mbar_wait(empty + stage, phase ^ 1u, abort_flag)) { ok = false; break; }
+                    if (lane == 0) {
+                        mbar_arrive_expect_tx(full + stage, kTileABytes + kUeTileBBytes);
+                        tma_load_2d(sA + stage * kTileABytes, &tmA, full + stage, kb * kBK, mb * kBM, pol_a);
+                        tma_load_3d(sB + stage * kUeTileBBytes, &tmB, full + stage, kb * kBK, nb * kUeBN, 0, pol_b);
+                    }
+                    __syncwarp();
+                    ++fills;
+                    if (++stage == kUeStages) { stage = 0; phase ^= 1u; }
+                }
+            }
+            if (lane == 0) {
+                const int first = fills > kUeStages ? fills - kUeStages : 0;
+                for (int i = first; i < fills; ++i)
+                    mbar_wait_drain(full + (i % kUeStages), static_cast<uint32_t>((i / kUeStages) & 1));
+            }
+            __syncwarp();
+        } else if (warp == 1) {
+            // ----------------------------------------------------------- MMA ----
+            int stage = 0, slot = 0, tiles_done = 0;
+            uint32_t phase = 0, sphase = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; ok && t < tiles; t += gridDim.x, ++tiles_done) {
+                // The accumulator is free once the epilogue has read the previous tile.
+                if (!mbar_wait(acc_empty, (tiles_done & 1) ^ 1u, abort_flag)) { ok = false; break; }
+                tc_fence_after();
+                for (int kb = 0; kb < nkb; ++kb) {
+                    const int j = kb % kUeSfGroup;  // byte of the scale words this K block uses
+                    const uint32_t sf_col = static_cast<uint32_t>(kUeAccCols + slot * kUeSfColsPerSlot);
+                    if (j == 0) {
+                        // Scale factors of this group of K blocks: shared memory -> TMEM.
+                        if (!mbar_wait(sf_full + slot, sphase, abort_flag)) { ok = false; break; }
+                        tc_fence_after();
+                        if (lane == 0) {
+                            const uint32_t sf_smem = smem_u32(sSF + slot * kUeSfSlotBytes);
+                            tmem_cp_sf_block(tmem_base + sf_col, sdesc_sf_block(sf_smem));
+                            tmem_cp_sf_block(tmem_base + sf_col + 4, sdesc_sf_block(sf_smem + kUeSfaBytes));
+                            tmem_cp_sf_block(tmem_base + sf_col + 8, sdesc_sf_block(sf_smem + kUeSfaBytes + 512));
+                        }
+                        __syncwarp();
+                    }
+                    if (!mbar_wait(full + stage, phase, abort_flag)) { ok = false; break; }
+                    tc_fence_after();
+                    if (lane == 0) {
+                        const uint32_t a_addr = smem_u32(sA + stage * kTileABytes);
+                        const uint32_t b_addr = smem_u32(sB + stage * kUeTileBBytes);
+                        const uint32_t idesc = idesc_e4m3_ue8m0(kBM, kUeBN, j, j);
+#pragma unroll
+                        for (int k = 0; k < kBK / 32; ++k)
+                            umma_f8_block_scaled(tmem_base, sdesc_kmajor_sw128(a_addr + k * 32),
+                                                 sdesc_kmajor_sw128(b_addr + k * 32), idesc, tmem_base + sf_col,
+                                                 tmem_base + sf_col + 4, (kb > 0 || k > 0) ? 1u : 0u);
+                        umma_commit(empty + stage);
+                        if (j == kUeSfGroup - 1 || kb == nkb - 1) umma_commit(sf_empty + slot);
+                        if (kb == nkb - 1) umma_commit(acc_full);
+                    }
+                    __syncwarp();
+                    if (++stage == kUeStages) { stage = 0; phase ^= 1u; }
+                    if (j == kUeSfGroup - 1 || kb == nkb - 1) {
+                        if (++slot == kUeSfSlots) { slot = 0; sphase ^= 1u; }
+                    }
+                }
+            }
+            if (lane == 0) {
+                umma_commit(done);
+                mbar_wait_drain(done, 0);
+            }
+            __syncwarp();
+        } else if (warp == 2) {
+            // ---------------------------------------------- scale loader ----
+            // Per K block: lane l copies sa rows m0+4l..m0+4l+3 (16 bytes) and
+            // lanes 0-1 the two sb values of the tile, asynchronously; the
+            // copies complete the slot's barrier when they land, so this warp
+            // only ever waits for a free slot.  Rows past M and blocks past
+            // N are zero-filled (and never used).
+            int slot = 0;
+            uint32_t rphase = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; ok && t < tiles; t += gridDim.x) {
+                int mb, nb;
+                raster_tile(t, p.m_blocks, p.n_blocks, p.raster, mb, nb);
+                const int r4 = mb * kBM + lane * 4;
+                const int left = p.M - r4;
+                const uint32_t sa_bytes = left >= 4 ? 16u : (left > 0 ? static_cast<uint32_t>(left) * 4u : 0u);
+                const int nbl = nb * (kUeBN / 128) + (lane & 1);
+                const bool nb_ok = nbl < p.nbn;
+                for (int kb = 0; kb < nkb; ++kb) {
+                    if (!mbar_wait(raw_empty + slot, rphase ^ 1u, abort_flag)) { ok = false; break; }
+                    const uint32_t dst = smem_u32(sRaw + slot * kUeRawFloats);
+                    const float* src = sa_bytes ? p.sa + static_cast<int64_t>(kb) * p.sa_stride + r4 : p.sa;
+                    cp_async_16(dst + lane * 16, src, sa_bytes);
+                    if (lane < 2)
+                        cp_async_4(dst + (kBM + lane) * 4, nb_ok ? p.sb + static_cast<int64_t>(nbl) * nkb + kb : p.sb,
+                                   nb_ok ? 4u : 0u);
+                    cp_async_arrive(raw_full + slot);
+                    if (++slot == kUeRawSlots) { slot = 0; rphase ^= 1u; }
+                }
+            }
+            asm volatile("cp.async.wait_all;" ::: "memory");
+        } else {
+            // -------------------------------------------- scale converter ----
+            // FP32 scales -> UE8M0 codes in the scale-factor layout: lane l
+            // writes line l of each block (A rows l + 32c, c < 4; B's two
+            // 128-column blocks).  Rows past M / blocks past N get code 127
+            // (a scale of 1) and only meet zero-filled operands.
+            int rslot = 0, sslot = 0;
+            uint32_t rphase = 0, sphase = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; ok && t < tiles; t += gridDim.x) {
+                int mb, nb;
+                raster_tile(t, p.m_blocks, p.n_blocks, p.raster, mb, nb);
+                const int m0 = mb * kBM;
+                const int nb0 = nb * (kUeBN / 128);
+                for (int kb0 = 0; kb0 < nkb; kb0 += kUeSfGroup) {
+                    // One slot holds kUeSfGroup K blocks: byte j of every word
+                    // is the code of K block kb0 + j (127 where the tile has
+                    // fewer K blocks left).
+                    if (!mbar_wait(sf_empty + sslot, sphase ^ 1u, abort_flag)) { ok = false; break; }
+                    uint32_t a[4] = {0u, 0u, 0u, 0u}, b0 = 0u, b1 = 0u;
+#pragma unroll 1
+                    for (int j = 0; j < kUeSfGroup; ++j) {
+                        uint32_t ca[4] = {127u, 127u, 127u, 127u}, cb0 = 127u, cb1 = 127u;
+                        if (kb0 + j < nkb) {
+                            if (!mbar_wait(raw_full + rslot, rphase, abort_flag)) { ok = false; break; }
+                            const float* raw = sRaw + rslot * kUeRawFloats;
+#pragma unroll
+                            for (int c = 0; c < 4; ++c)
+                                if (m0 + lane + 32 * c < p.M) ca[c] = ue8m0_code(raw[lane + 32 * c]);
+                            if (nb0 < p.nbn) cb0 = ue8m0_code(raw[kBM]);
+                            if (nb0 + 1 < p.nbn) cb1 = ue8m0_code(raw[kBM + 1]);
+                            __syncwarp();
+                            if (lane == 0) mbar_arrive(raw_empty + rslot);
+                            if (++rslot == kUeRawSlots) { rslot = 0; rphase ^= 1u; }
+                        }
+#pragma unroll
+                        for (int c = 0; c < 4; ++c) a[c] |= ca[c] << (8 * j);
+                        b0 |= cb0 << (8 * j);
+                        b1 |= cb1 << (8 * j);
+                    }
+                    if (!ok) break;
+                    const uint32_t base = smem_u32(sSF + sslot * kUeSfSlotBytes);
+                    st_shared_v4(base + lane * 16, a[0], a[1], a[2], a[3]);
+                    st_shared_v4(base + kUeSfaBytes + lane * 16, b0, b0, b0, b0);
+                    st_shared_v4(base + kUeSfaBytes + 512 + lane * 16, b1, b1, b1, b1);
+                    fence_proxy_async_smem();  // the copy to TMEM reads through the async proxy
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(sf_full + sslot);
+                    if (++sslot == kUeSfSlots) { sslot = 0; sphase ^= 1u; }
+                }
+            }
+        }
+    } else {
+        // ------------------------------------------------------- epilogue ----
+        regs_inc<224>();
+        const int ew = warp - kFirstEpiWarp;
+        const int half = ew >> 2;  // 128-column half of the tile
+        const int quarter = warp & 3;
+        const uint32_t t_lane = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16);
+        int tiles_done = 0;
+        bool ok = true;
+        for (int t = blockIdx.x; ok && t < tiles; t += gridDim.x, ++tiles_done) {
+            int mb, nb;
+            raster_tile(t, p.m_blocks, p.n_blocks, p.raster, mb, nb);
+            if (!mbar_wait(acc_full, tiles_done & 1, abort_flag)) { ok = false; break; }
+            tc_fence_after();
+            uint32_t v[4][32];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) tmem_ld_32x32b_x32(t_lane + static_cast<uint32_t>(half * 128 + c * 32), v[c]);
+            tmem_ld_wait();
+#pragma unroll
+            for (int c = 0; c < 4; ++c) reg_fence(v[c]);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(acc_empty);  // the MMA may start the next tile
+            // bf16, staged 32 rows x 32 columns at a time with the 64-byte
+            // swizzle of the output map, one TMA store per piece.
+            const uint32_t stg = smem_u32(sOut + ew * kStageOutBytes);
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                if (lane == 0) bulk_wait_read<0>();
+                __syncwarp();
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    uint32_t w4[4];
+#pragma unroll
+                    for (int h = 0; h < 4; ++h) {
+                        __nv_bfloat162 b = __floats2bfloat162_rn(__uint_as_float(v[c][q * 8 + 2 * h]),
+                                                                 __uint_as_float(v[c][q * 8 + 2 * h + 1]));
+                        w4[h] = *reinterpret_cast<uint32_t*>(&b);
+                    }
+                    const uint32_t off = lane * 64 + ((q ^ ((lane >> 1) & 3)) << 4);
+                    st_shared_v4(stg + off, w4[0], w4[1], w4[2], w4[3]);
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                const int x = nb * kUeBN + half * 128 + c * 32;
+                if (lane == 0 && x < p.N) {
+                    tma_store_2d(&tmD, sOut + ew * kStageOutBytes, x, mb * kBM + quarter * 32);
+                    bulk_commit();
+                }
+            }
+        }
+        if (lane == 0) bulk_wait<0>();
+        __syncwarp();
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, kUeTmemCols);
+    }
+}
+
+}  // namespace dg

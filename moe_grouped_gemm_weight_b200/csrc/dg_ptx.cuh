@@ -428,6 +428,45 @@ __host__ __device__ constexpr uint32_t idesc_e4m3_f32(int m, int n) {
     return (1u << 4) | (static_cast<uint32_t>(n >> 3) << 17) | (static_cast<uint32_t>(m >> 4) << 24);
 }
 
+// ------------------------------------------ block-scaled MMA (UE8M0) ----
+// Instruction descriptor of tcgen05.mma kind::mxf8f6f4.block_scale with e4m3
+// A and B (format 0), both K-major, UE8M0 scale factors (bit 23), M x N.
+// a_sf_id / b_sf_id pick the byte of each 32-bit scale-factor word this
+// K=32 step uses.  There is no accumulator-format field: it is FP32.
+__host__ __device__ constexpr uint32_t idesc_e4m3_ue8m0(int m, int n, int a_sf_id, int b_sf_id) {
+    return (static_cast<uint32_t>(b_sf_id & 3) << 4) | (static_cast<uint32_t>(n >> 3) << 17) | (1u << 23) |
+           (static_cast<uint32_t>(m >> 4) << 24) | (static_cast<uint32_t>(a_sf_id & 3) << 29);
+}
+
+// D(tmem) (+)= (A * 2^sfA)(smem) * (B * 2^sfB)(smem)^T over K = 32, the scale
+// factors read from TMEM at sfa_tmem / sfb_tmem.
+__device__ __forceinline__ void umma_f8_block_scaled(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                                     uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %6, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%4], [%5], p;\n\t}\n" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(sfa_tmem), "r"(sfb_tmem), "r"(accumulate)
+        : "memory");
+}
+
+// Shared-memory descriptor of a scale-factor block: 32 lines of 16 bytes,
+// contiguous, no swizzle (core matrices of 8 lines, 128 bytes apart).
+__device__ __forceinline__ uint64_t sdesc_sf_block(uint32_t saddr) {
+    uint64_t d = 0;
+    d |= static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4);
+    d |= static_cast<uint64_t>(128 >> 4) << 32;  // stride between 8-line core matrices
+    d |= static_cast<uint64_t>(1) << 46;         // descriptor version
+    return d;                                    // layout type 0: no swizzle
+}
+
+// Copy one scale-factor block (32 lines x 128 bits) from shared memory to
+// TMEM columns [col, col+4) of lanes 0-31, replicated to the four 32-lane
+// quarters.  Ordered with the issuing thread's later tcgen05.mma.
+__device__ __forceinline__ void tmem_cp_sf_block(uint32_t taddr, uint64_t sdesc) {
+    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
 // One UMMA: D(tmem) (+)= A(smem) * B(smem)^T, M x N x 32 for 8-bit inputs.
 __device__ __forceinline__ void umma_f8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
                                         uint32_t accumulate) {
