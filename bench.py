@@ -178,7 +178,7 @@ class Problem:
         if pl["swap_ab"]:
             self.kernel = f"fp8_gemm_swapab_kernel<{pl['block_m']}, {mode}>"
         else:
-            self.kernel = f"fp8_gemm_kernel<{pl['block_n']}, {pl['stages']}, {mode}>"
+            self.kernel = f"fp8_gemm_kernel<{pl['block_n']}, {pl['stages']}, {mode}, 0>"
 
     def run(self, case=None, D=None):
         c = case or self.case
@@ -335,6 +335,48 @@ def time_ue8m0(dg, launches: int, warmup: int, stream) -> list:
             row[f"us_{path}"] = round(t * 1e6, 2)
             row[f"tflops_{path}"] = round(pr.flops / t / 1e12, 1)
             del gr
+        out.append(row)
+    return out
+
+
+class LayoutProblem(Problem):
+    """A dense problem run with its operands stored in another order (the same
+    values, transposed copies): "nt", "nn", "tn" or "tt"."""
+
+    def __init__(self, case, dg, layout):
+        super().__init__(case, dg)
+        self.layout = layout
+        self.kernel = self.kernel.replace(", 0>", f", {dict(nt=0, tt=1, nn=2, tn=3)[layout]}>")
+
+    def run(self, case=None, D=None):
+        c = case or self.case
+        D = self.D if D is None else D
+        a_t, b_t = self.layout[0] == "t", self.layout[1] == "n"
+        key = (c.A.data_ptr(), c.B.data_ptr())
+        cache = self.__dict__.setdefault("_stored", {})
+        if key not in cache:  # transposed copies, made once per input copy (untimed warm-up)
+            cache[key] = (c.A.t().contiguous() if a_t else c.A, c.B.t().contiguous() if b_t else c.B)
+        A, B = cache[key]
+        getattr(self.dg, f"dg_fp8_gemm_{self.layout}")(D, A, c.sa, c.sa_stride, B, c.sb)
+
+
+LAYOUT_SHAPES = [(4096, 7168, 16384), (4096, 4096, 7168)]
+
+
+def time_layouts(dg, launches: int, warmup: int, stream) -> list:
+    out = []
+    for (m, n, k) in LAYOUT_SHAPES:
+        case = wl.dense_case(m, n, k, seed=0, device="cuda")
+        row = {"M": m, "N": n, "K": k}
+        for layout in ("nt", "nn", "tn", "tt"):
+            pr = LayoutProblem(case, dg, layout)
+            gr = RotatingGraph(pr, launches, warmup, stream)
+            gr.replay()
+            torch.cuda.synchronize()
+            t = gr.seconds_per_launch()
+            row[f"us_{layout}"] = round(t * 1e6, 2)
+            row[f"tflops_{layout}"] = round(pr.flops / t / 1e12, 1)
+            del gr, pr
         out.append(row)
     return out
 
@@ -542,6 +584,7 @@ def run_ours(args, rank, world, local):
 
     casts = [] if args.no_grouped else time_casts(dg, max(3, min(args.steps, 20)), args.warmup, cap_stream)
     ue8m0 = [] if args.no_grouped else time_ue8m0(dg, max(3, min(args.steps, 10)), args.warmup, cap_stream)
+    layouts = [] if args.no_grouped else time_layouts(dg, max(3, min(args.steps, 10)), args.warmup, cap_stream)
     for c in casts:
         c["frac_hbm_measured"] = round(c["gbs"] / peaks["hbm_gbs"], 3)
 
@@ -600,6 +643,7 @@ def run_ours(args, rank, world, local):
         "grouped": grouped_out,
         "cast": casts,
         "ue8m0": ue8m0,
+        "layouts": layouts,
         "roofline": roof,
         "cpu_baseline": cpu,
         "e2e": e2e,

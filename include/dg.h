@@ -96,6 +96,27 @@ DG_API dg_status dg_fp8_gemm_nt(uint16_t* D, const uint8_t* A, const float* sa, 
                          const uint8_t* B, const float* sb, int M, int N, int K, void* stream);
 
 /*
+ * Dense GEMM with the operands in the other storage orders.  The later-version
+ * article on DeepGEMM (section 3.1) notes that from SM100 on all four layouts
+ * NT, TN, NN and TT are supported.  The product is the same D = A . B^T with
+ * logical A [M][K] and B [N][K] and the same scales (sa transposed per 1x128,
+ * sb [ceil(N/128)][K/128]); only where A and B live changes:
+ *   dg_fp8_gemm_nn   A [M][K] (K contiguous),   B stored [K][N] (N contiguous)
+ *   dg_fp8_gemm_tn   A stored [K][M] (M contiguous), B stored [K][N]
+ *   dg_fp8_gemm_tt   A stored [K][M],           B [N][K] (K contiguous)
+ * (dg_fp8_gemm_nt is A [M][K], B [N][K].)  A stored [K][M] needs M % 16 == 0,
+ * B stored [K][N] needs N % 16 == 0 (16-byte rows for TMA); otherwise the
+ * limits of dg_fp8_gemm_nt hold.  These calls always use the 128 x {128,256}
+ * tile kernel (no few-row kernel).
+ */
+DG_API dg_status dg_fp8_gemm_nn(uint16_t* D, const uint8_t* A, const float* sa, int sa_stride,
+                                const uint8_t* B, const float* sb, int M, int N, int K, void* stream);
+DG_API dg_status dg_fp8_gemm_tn(uint16_t* D, const uint8_t* A, const float* sa, int sa_stride,
+                                const uint8_t* B, const float* sb, int M, int N, int K, void* stream);
+DG_API dg_status dg_fp8_gemm_tt(uint16_t* D, const uint8_t* A, const float* sa, int sa_stride,
+                                const uint8_t* B, const float* sb, int M, int N, int K, void* stream);
+
+/*
  * Dense GEMM for power-of-two scales, scaled inside the tensor core.  Same
  * arguments, layouts and result as dg_fp8_gemm_nt, but every sa and sb value
  * must be a positive normal power of two (UE8M0-representable: its FP32

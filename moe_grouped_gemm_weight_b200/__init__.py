@@ -56,6 +56,9 @@ def lib() -> ctypes.CDLL:
             P, I = ctypes.c_void_p, ctypes.c_int
             L.dg_fp8_gemm_nt.restype = I
             L.dg_fp8_gemm_nt.argtypes = [P, P, P, I, P, P, I, I, I, P]
+            for nm in ("dg_fp8_gemm_nn", "dg_fp8_gemm_tn", "dg_fp8_gemm_tt"):
+                getattr(L, nm).restype = I
+                getattr(L, nm).argtypes = [P, P, P, I, P, P, I, I, I, P]
             L.dg_fp8_gemm_nt_ue8m0.restype = I
             L.dg_fp8_gemm_nt_ue8m0.argtypes = [P, P, P, I, P, P, I, I, I, P]
             L.dg_fp8_gemm_nt_noalloc.restype = I
@@ -117,6 +120,30 @@ def dg_fp8_gemm_nt(D, A, sa, sa_stride: int, B, sb, stream=None) -> None:
     M, K = A.shape[-2], A.shape[-1]
     N = B.shape[-2]
     _check("dg_fp8_gemm_nt", lib().dg_fp8_gemm_nt(_ptr(D), _ptr(A), _ptr(sa), int(sa_stride), _ptr(B), _ptr(sb),
+                                                  M, N, K, _stream(stream)))
+
+
+def dg_fp8_gemm_nn(D, A, sa, sa_stride: int, B, sb, stream=None) -> None:
+    """D[M,N] = scaled A . B^T with A [M,K] and B stored [K,N]."""
+    M, K = A.shape[-2], A.shape[-1]
+    N = B.shape[-1]
+    _check("dg_fp8_gemm_nn", lib().dg_fp8_gemm_nn(_ptr(D), _ptr(A), _ptr(sa), int(sa_stride), _ptr(B), _ptr(sb),
+                                                  M, N, K, _stream(stream)))
+
+
+def dg_fp8_gemm_tn(D, A, sa, sa_stride: int, B, sb, stream=None) -> None:
+    """D[M,N] = scaled A . B^T with A stored [K,M] and B stored [K,N]."""
+    K, M = A.shape[-2], A.shape[-1]
+    N = B.shape[-1]
+    _check("dg_fp8_gemm_tn", lib().dg_fp8_gemm_tn(_ptr(D), _ptr(A), _ptr(sa), int(sa_stride), _ptr(B), _ptr(sb),
+                                                  M, N, K, _stream(stream)))
+
+
+def dg_fp8_gemm_tt(D, A, sa, sa_stride: int, B, sb, stream=None) -> None:
+    """D[M,N] = scaled A . B^T with A stored [K,M] and B [N,K]."""
+    K, M = A.shape[-2], A.shape[-1]
+    N = B.shape[-2]
+    _check("dg_fp8_gemm_tt", lib().dg_fp8_gemm_tt(_ptr(D), _ptr(A), _ptr(sa), int(sa_stride), _ptr(B), _ptr(sb),
                                                   M, N, K, _stream(stream)))
 
 

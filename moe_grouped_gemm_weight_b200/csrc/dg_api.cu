@@ -123,6 +123,22 @@ dg_status make_operand_map(CUtensorMap* tm, const void* base, int K, int rows, i
     return DG_OK;
 }
 
+// MN-major operand stored [K][MN] (MN contiguous, MN % 16 == 0): dims (MN, K),
+// box 128 (MN) x 128 (K) with 128-byte swizzle -- the canonical MN-major tile.
+dg_status make_mn_operand_map(CUtensorMap* tm, const void* base, int MN, int K) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return fail(DG_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(MN), static_cast<cuuint64_t>(K)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(MN)};
+    cuuint32_t box[2] = {128, static_cast<cuuint32_t>(dg::kBK)};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(DG_ERR_CUDA, "cuTensorMapEncodeTiled (MN-major) failed (CUresult %d)", static_cast<int>(r));
+    return DG_OK;
+}
+
 // bf16 output: dims (N, rows[, groups]), box (32, 32[, 1]) -- one promotion
 // warp's 32 rows x 32 columns -- with 64-byte swizzle; the store clips
 // everything outside the tensor.
@@ -177,13 +193,15 @@ constexpr int smem_for() {
 // the DeepGEMM README page (section "非对齐的块大小"); here BN stays a
 // multiple of 64 so that the two promotion warpgroups split it into 32-column
 // TMEM loads.
-Choice choose(int m_blocks, int pair_m_blocks, int N, int num_sms, bool pair_ok) {
+Choice choose(int m_blocks, int pair_m_blocks, int N, int num_sms, bool pair_ok, bool mn_major = false) {
     // 192 (three promotion warpgroups) is measured ~12% slower per tile than
-    // 256 on the dense sweep: reachable with DG_FORCE_BN, not chosen.
+    // 256 on the dense sweep: reachable with DG_FORCE_BN, not chosen.  An
+    // MN-major B is loaded in 128-wide atoms: tiles of 128 or 256 only.
     const int cands[3] = {256, 128, 64};
     Choice best{128, max_stages<128>(), false};
     double best_cost = -1.0;
     for (int bn : cands) {
+        if (mn_major && bn % 128 != 0) continue;
         const int tiles = m_blocks * cdiv(N, bn);
         const double t_kb = bn > 0.75 * (128 + bn) ? bn : 0.75 * (128 + bn);
         const double cost = static_cast<double>(waves_cost(tiles, num_sms)) * t_kb;
@@ -208,7 +226,7 @@ Choice choose(int m_blocks, int pair_m_blocks, int N, int num_sms, bool pair_ok)
     const char* force_bn = std::getenv("DG_FORCE_BN");
     if (force_bn && !best.pair) {
         const int f = std::atoi(force_bn);
-        if (f == 64 || f == 128 || f == 192 || f == 256) best.bn = f;
+        if (f == 128 || f == 256 || (!mn_major && (f == 64 || f == 192))) best.bn = f;
     }
     best.stages = best.pair ? kPairStages
                             : best.bn == 256 ? max_stages<256>()
@@ -258,12 +276,13 @@ int small_stages(int tn) {
     return tn == 32 ? dg::SmallCfg<32>::kStages : tn == 64 ? dg::SmallCfg<64>::kStages : dg::SmallCfg<128>::kStages;
 }
 
-dg_status plan(int mode, int rows, int N, int K, int G, int num_sms, dg_plan* out, int expected_m = 0) {
+dg_status plan(int mode, int rows, int N, int K, int G, int num_sms, dg_plan* out, int expected_m = 0,
+               int layout = 0) {
     dg_status s = check_sizes(mode, rows, N, K, G);
     if (s != DG_OK) return s;
     if (num_sms <= 0) return fail(DG_ERR_INVALID_ARG, "num_sms must be positive");
     *out = dg_plan{};
-    if (use_small(mode, rows)) {
+    if (layout == 0 && use_small(mode, rows)) {
         const int tn = small_tn(mode, rows);
         const int per_group = cdiv(rows, tn);
         const int m_blocks = mode == 2 ? G * per_group : per_group;
@@ -295,9 +314,9 @@ dg_status plan(int mode, int rows, int N, int K, int G, int num_sms, dg_plan* ou
     // CTA pairs are measured no faster than single-CTA 128 x 256 tiles on the
     // dense sweep, so they are used only when DG_FORCE_PAIR=1 (experiments).
     const char* force_pair = std::getenv("DG_FORCE_PAIR");
-    const bool pairs = force_pair && force_pair[0] == '1' && mode != 1;
+    const bool pairs = force_pair && force_pair[0] == '1' && mode != 1 && layout == 0;
     const int pair_m_blocks = (mode == 2 ? G : 1) * cdiv(rows, dg::kPairBM);
-    const Choice c = choose(m_blocks, pair_m_blocks, N, num_sms, pairs);
+    const Choice c = choose(m_blocks, pair_m_blocks, N, num_sms, pairs, layout != 0);
     if (c.pair) {
         const int per_group = cdiv(rows, dg::kPairBM);
         out->block_m = dg::kPairBM;
@@ -372,12 +391,12 @@ void set_pdl(cudaLaunchAttribute& a) {
     a.val.programmaticStreamSerializationAllowed = pdl_enabled() ? 1 : 0;
 }
 
-template <int BN, int STAGES, int MODE>
+template <int BN, int STAGES, int MODE, int LAYOUT = 0>
 dg_status launch_one(const dg::Params& p, const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& td,
                      int grid, cudaStream_t stream) {
     constexpr int smem = dg::smem_bytes<BN, STAGES>();
     static_assert(smem <= 227 * 1024, "shared memory budget exceeded");
-    auto kern = dg::fp8_gemm_kernel<BN, STAGES, MODE>;
+    auto kern = dg::fp8_gemm_kernel<BN, STAGES, MODE, LAYOUT>;
     static std::atomic<int> attr_set[kMaxDevices];
     int dev = 0;
     cudaGetDevice(&dev);
@@ -530,6 +549,16 @@ dg_status dispatch(const dg_plan& pl, const dg::Params& p, const CUtensorMap& ta
     }
 }
 
+template <int LAYOUT>
+dg_status dispatch_layout(const dg_plan& pl, const dg::Params& p, const CUtensorMap& ta, const CUtensorMap& tb,
+                          const CUtensorMap& td, cudaStream_t stream) {
+    switch (pl.block_n) {
+        case 256: return launch_one<256, max_stages<256>(), dg::kDense, LAYOUT>(p, ta, tb, td, pl.grid, stream);
+        case 128: return launch_one<128, max_stages<128>(), dg::kDense, LAYOUT>(p, ta, tb, td, pl.grid, stream);
+        default: return fail(DG_ERR_UNSUPPORTED, "no MN-major kernel for block_n=%d", pl.block_n);
+    }
+}
+
 int effective_sms() {
     const int dev_sms = device_sm_count();
     const int cap = g_num_sms_cap.load();
@@ -633,6 +662,46 @@ dg::Params make_params(uint16_t* D, const float* sa, int sa_stride, const float*
     p.tail_split = 1;
     p.full_tiles = pl.tiles;
     return p;
+}
+
+// Dense GEMM with the operands in any of the four storage orders (bit 0 of
+// `layout`: A stored [K][M]; bit 1: B stored [K][N]).
+dg_status gemm_layout(int layout, uint16_t* D, const uint8_t* A, const float* sa, int sa_stride, const uint8_t* B,
+                      const float* sb, int M, int N, int K, void* stream) {
+    dg_status s = check_sizes(0, M, N, K, 1);
+    if (s != DG_OK) return s;
+    if ((s = common_checks(D, A, sa, sa_stride, B, sb, M)) != DG_OK) return s;
+    if ((layout & 1) && M % 16 != 0) return fail(DG_ERR_UNSUPPORTED, "A stored [K][M] needs M %% 16 == 0 (M=%d)", M);
+    if ((layout & 2) && N % 16 != 0) return fail(DG_ERR_UNSUPPORTED, "B stored [K][N] needs N %% 16 == 0 (N=%d)", N);
+    if (M == 0) return ok();
+    const int sms = effective_sms();
+    if (sms <= 0) return fail(DG_ERR_CUDA, "no CUDA device");
+    dg_plan pl;
+    if ((s = plan(0, M, N, K, 1, sms, &pl, 0, layout)) != DG_OK) return s;
+    CUtensorMap ta, tb, td;
+    if ((s = (layout & 1) ? make_mn_operand_map(&ta, A, M, K) : make_operand_map(&ta, A, K, M, 1, dg::kBM, false)) !=
+        DG_OK)
+        return s;
+    if ((s = (layout & 2) ? make_mn_operand_map(&tb, B, N, K) : make_operand_map(&tb, B, K, N, 1, pl.block_n, true)) !=
+        DG_OK)
+        return s;
+    if ((s = make_output_map(&td, D, N, M, 1, false)) != DG_OK) return s;
+    dg::Params p = make_params(D, sa, sa_stride, sb, M, N, K, 1, pl);
+    p.b_stream = pl.m_blocks == 1;
+    TailWorkspace ws;
+    if (pl.tail_split > 1 && tail_workspace(static_cast<cudaStream_t>(stream), &ws)) {
+        p.tail_split = pl.tail_split;
+        p.full_tiles = (pl.tiles / pl.grid) * pl.grid;
+        p.ws = ws.partials;
+        p.ws_flags = ws.flags;
+    }
+    const cudaStream_t st = static_cast<cudaStream_t>(stream);
+    switch (layout) {
+        case 1: return dispatch_layout<1>(pl, p, ta, tb, td, st);
+        case 2: return dispatch_layout<2>(pl, p, ta, tb, td, st);
+        case 3: return dispatch_layout<3>(pl, p, ta, tb, td, st);
+        default: return fail(DG_ERR_INVALID_ARG, "bad layout %d", layout);
+    }
 }
 
 }  // namespace
@@ -831,6 +900,21 @@ dg_status dg_fp8_gemm_nt_ue8m0(uint16_t* D, const uint8_t* A, const float* sa, i
     if (e == cudaSuccess) e = cudaGetLastError();
     if (e != cudaSuccess) return fail(DG_ERR_CUDA, "kernel launch failed: %s", cudaGetErrorString(e));
     return ok();
+}
+
+dg_status dg_fp8_gemm_nn(uint16_t* D, const uint8_t* A, const float* sa, int sa_stride, const uint8_t* B,
+                         const float* sb, int M, int N, int K, void* stream) {
+    return gemm_layout(2, D, A, sa, sa_stride, B, sb, M, N, K, stream);
+}
+
+dg_status dg_fp8_gemm_tn(uint16_t* D, const uint8_t* A, const float* sa, int sa_stride, const uint8_t* B,
+                         const float* sb, int M, int N, int K, void* stream) {
+    return gemm_layout(3, D, A, sa, sa_stride, B, sb, M, N, K, stream);
+}
+
+dg_status dg_fp8_gemm_tt(uint16_t* D, const uint8_t* A, const float* sa, int sa_stride, const uint8_t* B,
+                         const float* sb, int M, int N, int K, void* stream) {
+    return gemm_layout(1, D, A, sa, sa_stride, B, sb, M, N, K, stream);
 }
 
 dg_status dg_grouped_contiguous_nt(uint16_t* D, const uint8_t* A, const float* sa, int sa_stride, const uint8_t* B,

@@ -183,12 +183,19 @@ __device__ __forceinline__ Tile decode_tile(const Params& p, int t, int m_blocks
     return tl;
 }
 
-template <int BN, int STAGES, int MODE>
+// LAYOUT (dense only) gives the operands' storage: bit 0 set = A stored
+// [K][M] (M-major, the "T" of TN / TT), bit 1 set = B stored [K][N] (N-major,
+// the "N" of NN / TN); clear = K-major as in NT.  An MN-major operand is loaded
+// as 128 x 128 TMA boxes (MN inner) and described to the MMA as MN-major.
+template <int BN, int STAGES, int MODE, int LAYOUT = 0>
 __global__ void __launch_bounds__(Cfg<BN>::kThreadsC, 1)
 fp8_gemm_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtensorMap tmA,
                 const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmD) {
     using C = Cfg<BN>;
     constexpr int kNBuf = C::kNBuf;
+    constexpr bool kAmn = (LAYOUT & 1) != 0;
+    constexpr bool kBmn = (LAYOUT & 2) != 0;
+    static_assert(LAYOUT == 0 || (MODE == kDense && BN % 128 == 0), "MN-major operands: dense, BN 128 or 256");
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -299,11 +306,20 @@ fp8_gemm_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtens
                 if (!mbar_wait(empty + stage, phase ^ 1u, abort_flag)) { ok = false; break; }
                 if (lane == 0) {
                     mbar_arrive_expect_tx(full + stage, kTileABytes + C::kTileBBytes);
-                    if (MODE == kMasked)
+                    if (kAmn)
+                        tma_load_2d(sA + stage * kTileABytes, &tmA, full + stage, tl.m0, kb * kBK, pol_a);
+                    else if (MODE == kMasked)
                         tma_load_3d(sA + stage * kTileABytes, &tmA, full + stage, kb * kBK, tl.m0, tl.g, pol_a);
                     else
                         tma_load_2d(sA + stage * kTileABytes, &tmA, full + stage, kb * kBK, tl.m0, pol_a);
-                    tma_load_3d(sB + stage * C::kTileBBytes, &tmB, full + stage, kb * kBK, tl.n0, tl.g, pol_b);
+                    if (kBmn) {
+#pragma unroll
+                        for (int h = 0; h < BN / 128; ++h)
+                            tma_load_2d(sB + stage * C::kTileBBytes + h * 128 * kBK, &tmB, full + stage, tl.n0 + h * 128,
+                                        kb * kBK, pol_b);
+                    } else {
+                        tma_load_3d(sB + stage * C::kTileBBytes, &tmB, full + stage, kb * kBK, tl.n0, tl.g, pol_b);
+                    }
                 }
                 __syncwarp();
                 ++fills;
@@ -320,7 +336,7 @@ fp8_gemm_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtens
         __syncwarp();
     } else if (warp == 1) {
         // ----------------------------------------------------------- MMA ----
-        constexpr uint32_t idesc = idesc_e4m3_f32(kBM, BN);
+        constexpr uint32_t idesc = idesc_e4m3_f32_major(kBM, BN, kAmn, kBmn);
         int stage = 0, buf = 0;
         uint32_t phase = 0, bphase = 0;
         bool ok = true;
@@ -337,9 +353,13 @@ fp8_gemm_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtens
                     const uint32_t b_addr = smem_u32(sB + stage * C::kTileBBytes);
                     const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * BN);
 #pragma unroll
-                    for (int k = 0; k < kBK / 32; ++k)
-                        umma_f8(d_tmem, sdesc_kmajor_sw128(a_addr + k * 32), sdesc_kmajor_sw128(b_addr + k * 32),
-                                idesc, k > 0 ? 1u : 0u);
+                    for (int k = 0; k < kBK / 32; ++k) {
+                        const uint64_t ad = kAmn ? sdesc_mnmajor_sw128(a_addr + k * 32 * 128, 128 * kBK)
+                                                 : sdesc_kmajor_sw128(a_addr + k * 32);
+                        const uint64_t bd = kBmn ? sdesc_mnmajor_sw128(b_addr + k * 32 * 128, 128 * kBK)
+                                                 : sdesc_kmajor_sw128(b_addr + k * 32);
+                        umma_f8(d_tmem, ad, bd, idesc, k > 0 ? 1u : 0u);
+                    }
                     umma_commit(empty + stage);
                     umma_commit(tfull + buf);
                 }

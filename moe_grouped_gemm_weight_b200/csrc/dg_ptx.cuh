@@ -467,6 +467,27 @@ __device__ __forceinline__ void tmem_cp_sf_block(uint32_t taddr, uint64_t sdesc)
     asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
 }
 
+// Shared-memory descriptor of an MN-major operand tile loaded by TMA with the
+// 128-byte swizzle: each K row holds 128 MN elements (128 bytes), K rows are
+// 128 bytes apart, groups of 8 rows 1024 bytes apart (stride field), and
+// successive 128-element MN atoms `lbo_bytes` apart (leading field).  The
+// K=32 step of an MMA advances the start by 32 rows = 4096 bytes.
+__device__ __forceinline__ uint64_t sdesc_mnmajor_sw128(uint32_t saddr, uint32_t lbo_bytes) {
+    uint64_t d = 0;
+    d |= static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4);
+    d |= static_cast<uint64_t>((lbo_bytes >> 4) & 0x3FFFu) << 16;
+    d |= static_cast<uint64_t>(1024 >> 4) << 32;
+    d |= static_cast<uint64_t>(1) << 46;
+    d |= static_cast<uint64_t>(2) << 61;
+    return d;
+}
+
+// idesc_e4m3_f32 with the operands' majors: bit 15 A (1 = M-major), bit 16 B
+// (1 = N-major); valid for e4m3.
+__host__ __device__ constexpr uint32_t idesc_e4m3_f32_major(int m, int n, bool a_mn, bool b_mn) {
+    return idesc_e4m3_f32(m, n) | (a_mn ? (1u << 15) : 0u) | (b_mn ? (1u << 16) : 0u);
+}
+
 // One UMMA: D(tmem) (+)= A(smem) * B(smem)^T, M x N x 32 for 8-bit inputs.
 __device__ __forceinline__ void umma_f8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
                                         uint32_t accumulate) {
