@@ -381,6 +381,49 @@ def time_layouts(dg, launches: int, warmup: int, stream) -> list:
     return out
 
 
+# K-grouped GEMM (MoE weight gradient): experts x tokens per expert, M x N.
+KGROUPED = {"M": 7168, "N": 2048, "tokens": [4096, 4096, 4096, 4096]}
+
+
+def time_k_grouped(dg, launches: int, warmup: int, stream) -> dict:
+    """The K-grouped GEMM as a CUDA graph over input copies larger than L2."""
+    M, N, counts = KGROUPED["M"], KGROUPED["N"], KGROUPED["tokens"]
+    K = sum(counts)
+    case = wl.dense_case(M, N, K, seed=0, device="cuda")
+    offsets = torch.tensor([0] + list(torch.tensor(counts).cumsum(0).tolist()), dtype=torch.int32, device="cuda")
+    G = len(counts)
+    footprint = 2 * M * K + N * K + 2 * G * M * N
+    copies = min(64, max(2, -(-ROTATE_FACTOR * L2_BYTES // footprint)))
+    reps = [(case.A.t().contiguous(), case.B.t().contiguous(),
+             torch.empty(G, M, N, dtype=torch.bfloat16, device="cuda")) for _ in range(copies)]
+
+    def call(i):
+        At, Bt, D = reps[i % copies]
+        dg.dg_k_grouped_fp8_gemm_tn(D, At, case.sa, case.sa_stride, Bt, case.sb, offsets)
+
+    with torch.cuda.stream(stream):
+        for i in range(max(warmup, 1) * copies):
+            call(i)
+    stream.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        for i in range(launches):
+            call(i)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        graph.replay()
+        e0.record(stream)
+        graph.replay()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    t = e0.elapsed_time(e1) * 1e-3 / launches
+    flops = 2.0 * M * N * K
+    nbytes = M * K + N * K + 2 * G * M * N + 4 * M * (K // 128) + 4 * (-(-N // 128)) * (K // 128)
+    del graph, reps
+    return {"workload": f"K-grouped (weight gradient) G={G} tokens={counts} M={M} N={N}", "us": round(t * 1e6, 2),
+            "tflops": round(flops / t / 1e12, 1), "gbs": round(nbytes / t / 1e9, 1), "input_copies": copies}
+
+
 # FP8 cast workloads: (kind, rows, K); "1x128" = activations, "128x128" = weights.
 CAST_SHAPES = [("1x128", 4096, 7168), ("1x128", 32768, 7168), ("1x128", 128, 7168), ("1x128", 64, 7168),
                ("128x128", 7168, 16384), ("128x128", 4096, 7168)]
@@ -585,6 +628,9 @@ def run_ours(args, rank, world, local):
     casts = [] if args.no_grouped else time_casts(dg, max(3, min(args.steps, 20)), args.warmup, cap_stream)
     ue8m0 = [] if args.no_grouped else time_ue8m0(dg, max(3, min(args.steps, 10)), args.warmup, cap_stream)
     layouts = [] if args.no_grouped else time_layouts(dg, max(3, min(args.steps, 10)), args.warmup, cap_stream)
+    kgrouped = None if args.no_grouped else time_k_grouped(dg, max(3, min(args.steps, 10)), args.warmup, cap_stream)
+    if kgrouped:
+        kgrouped["frac_roof_measured"] = round(kgrouped["tflops"] / p_fp8_sust, 3)
     for c in casts:
         c["frac_hbm_measured"] = round(c["gbs"] / peaks["hbm_gbs"], 3)
 
@@ -644,6 +690,7 @@ def run_ours(args, rank, world, local):
         "cast": casts,
         "ue8m0": ue8m0,
         "layouts": layouts,
+        "k_grouped": kgrouped,
         "roofline": roof,
         "cpu_baseline": cpu,
         "e2e": e2e,

@@ -81,6 +81,8 @@ typedef enum dg_status {
 #define DG_DEVERR_BAD_MASKED_M 4u   /* masked: masked_m value not in [0,M_max]  */
 #define DG_DEVERR_NOT_POW2 8u       /* ue8m0 call: a scale is not a positive     */
                                     /* normal power of two                       */
+#define DG_DEVERR_BAD_K_OFFSET 16u  /* K-grouped: k_offsets not increasing       */
+                                    /* multiples of 128 within [0, K]            */
 
 /*
  * Dense GEMM: D[M,N] = scaled A[M,K] . B[N,K]^T (section "常规密集型 GEMM（非分组）",
@@ -115,6 +117,28 @@ DG_API dg_status dg_fp8_gemm_tn(uint16_t* D, const uint8_t* A, const float* sa, 
                                 const uint8_t* B, const float* sb, int M, int N, int K, void* stream);
 DG_API dg_status dg_fp8_gemm_tt(uint16_t* D, const uint8_t* A, const float* sa, int sa_stride,
                                 const uint8_t* B, const float* sb, int M, int N, int K, void* stream);
+
+/*
+ * Grouped GEMM along K (the weight-gradient GEMM of a MoE layer; the
+ * later-version article on DeepGEMM, section 3.2, names grouping along M or
+ * along K).  Group g owns the K rows [k_offsets[g], k_offsets[g+1]) -- e.g.
+ * the tokens routed to expert g -- and
+ *   D[g][m][n] = bf16( sum over g's K blocks kb of sa[m,kb]*sb[n/128,kb]*P_kb[m,n] ),
+ * the dense formula restricted to the group's K blocks (an empty group gives
+ * zeros).  Storage as in dg_fp8_gemm_tn, with K the total over all groups:
+ *   A          uint8 e4m3 stored [K][M] (M contiguous, M % 16 == 0)
+ *   B          uint8 e4m3 stored [K][N] (N contiguous, N % 16 == 0)
+ *   sa         float32, sa[kb*sa_stride + m], kb < K/128 (global K blocks)
+ *   sb         float32 [ceil(N/128)][K/128]
+ *   k_offsets  int32 [G+1] on the device, increasing multiples of 128 with
+ *              k_offsets[G] <= K; bad values set DG_DEVERR_BAD_K_OFFSET and the
+ *              group's D is written as zeros
+ *   D          bf16 [G][M][N]
+ * M == 0 is valid and launches nothing.
+ */
+DG_API dg_status dg_k_grouped_fp8_gemm_tn(uint16_t* D, const uint8_t* A, const float* sa, int sa_stride,
+                                          const uint8_t* B, const float* sb, const int32_t* k_offsets, int G,
+                                          int M, int N, int K, void* stream);
 
 /*
  * Dense GEMM for power-of-two scales, scaled inside the tensor core.  Same

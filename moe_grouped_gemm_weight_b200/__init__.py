@@ -25,6 +25,7 @@ LIB_PATH = os.path.join(_HERE, "libdg.so")
 
 DG_OK, DG_ERR_INVALID_ARG, DG_ERR_UNSUPPORTED, DG_ERR_MISALIGNED, DG_ERR_CUDA = range(5)
 DG_DEVERR_TIMEOUT, DG_DEVERR_BAD_M_INDEX, DG_DEVERR_BAD_MASKED_M, DG_DEVERR_NOT_POW2 = 1, 2, 4, 8
+DG_DEVERR_BAD_K_OFFSET = 16
 
 _lock = threading.Lock()
 _lib = None
@@ -59,6 +60,8 @@ def lib() -> ctypes.CDLL:
             for nm in ("dg_fp8_gemm_nn", "dg_fp8_gemm_tn", "dg_fp8_gemm_tt"):
                 getattr(L, nm).restype = I
                 getattr(L, nm).argtypes = [P, P, P, I, P, P, I, I, I, P]
+            L.dg_k_grouped_fp8_gemm_tn.restype = I
+            L.dg_k_grouped_fp8_gemm_tn.argtypes = [P, P, P, I, P, P, P, I, I, I, I, P]
             L.dg_fp8_gemm_nt_ue8m0.restype = I
             L.dg_fp8_gemm_nt_ue8m0.argtypes = [P, P, P, I, P, P, I, I, I, P]
             L.dg_fp8_gemm_nt_noalloc.restype = I
@@ -145,6 +148,17 @@ def dg_fp8_gemm_tt(D, A, sa, sa_stride: int, B, sb, stream=None) -> None:
     N = B.shape[-2]
     _check("dg_fp8_gemm_tt", lib().dg_fp8_gemm_tt(_ptr(D), _ptr(A), _ptr(sa), int(sa_stride), _ptr(B), _ptr(sb),
                                                   M, N, K, _stream(stream)))
+
+
+def dg_k_grouped_fp8_gemm_tn(D, A, sa, sa_stride: int, B, sb, k_offsets, stream=None) -> None:
+    """K-grouped GEMM: A stored [K,M], B stored [K,N], k_offsets int32 [G+1] on the
+    device, D [G,M,N]."""
+    K, M = A.shape[-2], A.shape[-1]
+    N = B.shape[-1]
+    G = k_offsets.numel() - 1
+    _check("dg_k_grouped_fp8_gemm_tn",
+           lib().dg_k_grouped_fp8_gemm_tn(_ptr(D), _ptr(A), _ptr(sa), int(sa_stride), _ptr(B), _ptr(sb),
+                                          _ptr(k_offsets), G, M, N, K, _stream(stream)))
 
 
 def dg_fp8_gemm_nt_ue8m0(D, A, sa, sa_stride: int, B, sb, stream=None) -> None:

@@ -251,7 +251,7 @@ dg_status check_sizes(int mode, int rows, int N, int K, int G) {
     if (mode == 2 && G > dg::kMaxMaskedGroups)
         return fail(DG_ERR_UNSUPPORTED, "masked layout supports at most %d groups (G=%d)", dg::kMaxMaskedGroups, G);
     const long long a_elems = static_cast<long long>(rows) * K * (mode == 2 ? G : 1);
-    const long long b_elems = static_cast<long long>(G) * N * K;
+    const long long b_elems = static_cast<long long>(mode == 3 ? 1 : G) * N * K;
     if (a_elems >= (1ll << 40) || b_elems >= (1ll << 40) || static_cast<long long>(rows) * G >= (1ll << 31))
         return fail(DG_ERR_UNSUPPORTED, "problem too large");
     return DG_OK;
@@ -704,6 +704,49 @@ dg_status gemm_layout(int layout, uint16_t* D, const uint8_t* A, const float* sa
     }
 }
 
+// K-grouped GEMM (A stored [K][M], B stored [K][N], group g owning K rows
+// [k_offsets[g], k_offsets[g+1]), output D [G][M][N]).
+dg_status k_grouped(uint16_t* D, const uint8_t* A, const float* sa, int sa_stride, const uint8_t* B,
+                    const float* sb, const int32_t* k_offsets, int G, int M, int N, int K, void* stream) {
+    if (G <= 0 || M < 0 || N <= 0 || K <= 0)
+        return fail(DG_ERR_INVALID_ARG, "sizes must be positive (G=%d M=%d N=%d K=%d)", G, M, N, K);
+    dg_status s = check_sizes(3, M, N, K, G);
+    if (s != DG_OK) return s;
+    if ((s = common_checks(D, A, sa, sa_stride, B, sb, M)) != DG_OK) return s;
+    if (!k_offsets) return fail(DG_ERR_INVALID_ARG, "null k_offsets");
+    if (M % 16 != 0) return fail(DG_ERR_UNSUPPORTED, "A stored [K][M] needs M %% 16 == 0 (M=%d)", M);
+    if (N % 16 != 0) return fail(DG_ERR_UNSUPPORTED, "B stored [K][N] needs N %% 16 == 0 (N=%d)", N);
+    if (static_cast<long long>(G) * M >= (1ll << 31)) return fail(DG_ERR_UNSUPPORTED, "problem too large");
+    if (M == 0) return ok();
+    const int sms = effective_sms();
+    if (sms <= 0) return fail(DG_ERR_CUDA, "no CUDA device");
+    const int m_blocks = cdiv(M, dg::kBM);
+    const Choice c = choose(G * m_blocks, 0, N, sms, false, true);
+    dg_plan pl{};
+    pl.block_m = dg::kBM;
+    pl.block_n = c.bn;
+    pl.stages = c.stages;
+    pl.m_blocks = m_blocks;
+    pl.n_blocks = cdiv(N, c.bn);
+    pl.tiles = G * m_blocks * pl.n_blocks;
+    pl.grid = pl.tiles < sms ? pl.tiles : sms;
+    pl.smem_bytes = plan_smem(c);
+    pl.split_k = 1;
+    pl.tail_split = 1;
+    CUtensorMap ta, tb, td;
+    if ((s = make_mn_operand_map(&ta, A, M, K)) != DG_OK) return s;
+    if ((s = make_mn_operand_map(&tb, B, N, K)) != DG_OK) return s;
+    if ((s = make_output_map(&td, D, N, M, G, true)) != DG_OK) return s;
+    dg::Params p = make_params(D, sa, sa_stride, sb, M, N, K, G, pl);
+    p.k_offsets = k_offsets;
+    const cudaStream_t st = static_cast<cudaStream_t>(stream);
+    switch (pl.block_n) {
+        case 256: return launch_one<256, max_stages<256>(), dg::kKGrouped, 3>(p, ta, tb, td, pl.grid, st);
+        case 128: return launch_one<128, max_stages<128>(), dg::kKGrouped, 3>(p, ta, tb, td, pl.grid, st);
+        default: return fail(DG_ERR_UNSUPPORTED, "no K-grouped kernel for block_n=%d", pl.block_n);
+    }
+}
+
 }  // namespace
 
 // ------------------------------------------------ allocation-free dense ----
@@ -915,6 +958,12 @@ dg_status dg_fp8_gemm_tn(uint16_t* D, const uint8_t* A, const float* sa, int sa_
 dg_status dg_fp8_gemm_tt(uint16_t* D, const uint8_t* A, const float* sa, int sa_stride, const uint8_t* B,
                          const float* sb, int M, int N, int K, void* stream) {
     return gemm_layout(1, D, A, sa, sa_stride, B, sb, M, N, K, stream);
+}
+
+dg_status dg_k_grouped_fp8_gemm_tn(uint16_t* D, const uint8_t* A, const float* sa, int sa_stride, const uint8_t* B,
+                                   const float* sb, const int32_t* k_offsets, int G, int M, int N, int K,
+                                   void* stream) {
+    return k_grouped(D, A, sa, sa_stride, B, sb, k_offsets, G, M, N, K, stream);
 }
 
 dg_status dg_grouped_contiguous_nt(uint16_t* D, const uint8_t* A, const float* sa, int sa_stride, const uint8_t* B,

@@ -33,7 +33,7 @@
 
 namespace dg {
 
-enum Mode : int { kDense = 0, kContiguous = 1, kMasked = 2 };
+enum Mode : int { kDense = 0, kContiguous = 1, kMasked = 2, kKGrouped = 3 };
 
 constexpr int kBM = 128;                 // tile rows = tcgen05 M
 constexpr int kBK = 128;                 // K per block = scale granularity
@@ -52,6 +52,7 @@ struct Params {
     const float* sb;
     const int32_t* m_indices;  // contiguous mode
     const int32_t* masked_m;   // masked mode
+    const int32_t* k_offsets;  // K-grouped mode: group g owns K [k_offsets[g], k_offsets[g+1])
     int sa_stride;
     int M;          // dense: M; contiguous: M_total; masked: M_max
     int N, K, G;
@@ -155,6 +156,17 @@ __device__ __forceinline__ void raster_tile(int t, int m_blocks, int n_blocks, i
 template <int BN, int MODE>
 __device__ __forceinline__ Tile decode_tile(const Params& p, int t, int m_blocks, const int* mb_prefix) {
     int mb, nb;
+    if (MODE == kKGrouped) {
+        // Groups outermost: tiles of one group share its K range of A and B.
+        const int per_group = m_blocks * p.n_blocks;
+        raster_tile(t % per_group, m_blocks, p.n_blocks, p.raster, mb, nb);
+        Tile tl;
+        tl.g = t / per_group;
+        tl.m0 = mb * kBM;
+        tl.n0 = nb * BN;
+        tl.valid = true;
+        return tl;
+    }
     raster_tile(t, m_blocks, p.n_blocks, p.raster, mb, nb);
     Tile tl;
     tl.n0 = nb * BN;
@@ -183,6 +195,23 @@ __device__ __forceinline__ Tile decode_tile(const Params& p, int t, int m_blocks
     return tl;
 }
 
+// K-grouped mode: the tile's K blocks are its group's [k_offsets[g], k_offsets[g+1]).
+// Offsets that are not multiples of 128, decrease, or leave [0, K] are bad
+// data: flagged (DG_DEVERR_BAD_K_OFFSET) and the group treated as empty, so
+// its D is written as zeros.
+template <int MODE>
+__device__ __forceinline__ void group_k_range(const Params& p, const Tile& tl, Work& w) {
+    if (MODE != kKGrouped) return;
+    const int k0 = __ldg(p.k_offsets + tl.g), k1 = __ldg(p.k_offsets + tl.g + 1);
+    if (k0 < 0 || k1 < k0 || k1 > p.K || (k0 | k1) % kBK != 0) {
+        if (threadIdx.x == 0 && tl.m0 == 0 && tl.n0 == 0) atomicOr(&g_dg_error, 16u);
+        w.kb0 = w.kb1 = 0;
+        return;
+    }
+    w.kb0 = k0 / kBK;
+    w.kb1 = k1 / kBK;
+}
+
 // LAYOUT (dense only) gives the operands' storage: bit 0 set = A stored
 // [K][M] (M-major, the "T" of TN / TT), bit 1 set = B stored [K][N] (N-major,
 // the "N" of NN / TN); clear = K-major as in NT.  An MN-major operand is loaded
@@ -195,7 +224,9 @@ fp8_gemm_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtens
     constexpr int kNBuf = C::kNBuf;
     constexpr bool kAmn = (LAYOUT & 1) != 0;
     constexpr bool kBmn = (LAYOUT & 2) != 0;
-    static_assert(LAYOUT == 0 || (MODE == kDense && BN % 128 == 0), "MN-major operands: dense, BN 128 or 256");
+    static_assert(LAYOUT == 0 || ((MODE == kDense || MODE == kKGrouped) && BN % 128 == 0),
+                  "MN-major operands: dense or K-grouped, BN 128 or 256");
+    static_assert(MODE != kKGrouped || LAYOUT == 3, "K-grouped: A stored [K][M], B stored [K][N]");
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -282,7 +313,7 @@ fp8_gemm_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtens
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
     if (MODE == kMasked) m_blocks = mb_prefix[p.G];
-    const int tiles = m_blocks * p.n_blocks;
+    const int tiles = (MODE == kKGrouped ? p.G : 1) * m_blocks * p.n_blocks;
     const int nkb = p.nkb;
 
     // Register budget: the producer / MMA / scale warps need few registers,
@@ -302,6 +333,7 @@ fp8_gemm_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtens
         for (int it = 0; ok && next_work(p, tiles, it, w); ++it) {
             const Tile tl = decode_tile<BN, MODE>(p, w.t, m_blocks, mb_prefix);
             if (!tl.valid) continue;
+            group_k_range<MODE>(p, tl, w);
             for (int kb = w.kb0; kb < w.kb1; ++kb) {
                 if (!mbar_wait(empty + stage, phase ^ 1u, abort_flag)) { ok = false; break; }
                 if (lane == 0) {
@@ -344,6 +376,7 @@ fp8_gemm_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtens
         for (int it = 0; ok && next_work(p, tiles, it, w); ++it) {
             const Tile tl = decode_tile<BN, MODE>(p, w.t, m_blocks, mb_prefix);
             if (!tl.valid) continue;
+            group_k_range<MODE>(p, tl, w);
             for (int kb = w.kb0; kb < w.kb1; ++kb) {
                 if (!mbar_wait(tempty + buf, bphase ^ 1u, abort_flag)) { ok = false; break; }
                 if (!mbar_wait(full + stage, phase, abort_flag)) { ok = false; break; }
@@ -388,8 +421,9 @@ fp8_gemm_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtens
         for (int it = 0; next_work(p, tiles, it, w); ++it) {
             const Tile tl = decode_tile<BN, MODE>(p, w.t, m_blocks, mb_prefix);
             if (!tl.valid) continue;
+            group_k_range<MODE>(p, tl, w);
             const float* sa_base = p.sa + (MODE == kMasked ? static_cast<int64_t>(tl.g) * nkb * p.sa_stride : 0);
-            const float* sb_g = p.sb + static_cast<int64_t>(tl.g) * p.nbn * nkb;
+            const float* sb_g = p.sb + (MODE == kKGrouped ? 0 : static_cast<int64_t>(tl.g) * p.nbn * nkb);
             const int nb = tl.n0 / 128 + (lane & 3);
             const bool nb_ok = nb < p.nbn;
             const int r4 = tl.m0 + lane * 4;
@@ -428,6 +462,7 @@ fp8_gemm_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtens
         for (int it = 0; ok && next_work(p, tiles, it, w); ++it) {
             const Tile tl = decode_tile<BN, MODE>(p, w.t, m_blocks, mb_prefix);
             if (!tl.valid) continue;
+            group_k_range<MODE>(p, tl, w);
             const int g = tl.g;
             // Row validity and the row's output address.
             const int row = tl.m0 + r;
@@ -442,6 +477,9 @@ fp8_gemm_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtens
                 row_ok = (gi == g);
                 if (gi != g && gi != -1) atomicOr(&g_dg_error, 2u);
                 d_row = row;
+            } else if (MODE == kKGrouped) {
+                row_ok = row < p.M;
+                d_row = static_cast<int64_t>(g) * p.M + row;
             } else {
                 row_ok = row < p.M;
                 d_row = row;
@@ -553,7 +591,7 @@ fp8_gemm_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtens
             // one lane issues a TMA store; the copy drains while the warp
             // moves on.  Warps holding rows that must stay untouched (padding
             // rows, rows past masked_m) store their valid rows directly.
-            const bool clip_ok = row_ok || MODE == kDense || (MODE == kMasked && row >= p.M);
+            const bool clip_ok = row_ok || MODE == kDense || MODE == kKGrouped || (MODE == kMasked && row >= p.M);
             if (__all_sync(0xffffffffu, clip_ok)) {
                 const uint32_t stg = smem_u32(sOut + ew * kStageOutBytes);
 #pragma unroll
@@ -574,7 +612,7 @@ fp8_gemm_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtens
                     __syncwarp();
                     const int x = tl.n0 + col0 + pc * 32;
                     if (lane == 0 && x < p.N) {
-                        if (MODE == kMasked)
+                        if (MODE == kMasked || MODE == kKGrouped)
                             tma_store_3d(&tmD, sOut + ew * kStageOutBytes, x, tl.m0 + quarter * 32, g);
                         else
                             tma_store_2d(&tmD, sOut + ew * kStageOutBytes, x, tl.m0 + quarter * 32);
