@@ -192,10 +192,11 @@ class Problem:
 
 
 def kernel_source_sha() -> str:
-    import glob
+    """Hash of the device code that defines the dominant kernel instance (the
+    persistent GEMM kernel and the PTX helpers it uses)."""
     import hashlib
     h = hashlib.sha256()
-    for f in sorted(glob.glob(os.path.join(ROOT, "moe_grouped_gemm_weight_b200", "csrc", "*"))):
+    for f in [os.path.join(ROOT, "moe_grouped_gemm_weight_b200", "csrc", n) for n in ("dg_kernel.cuh", "dg_ptx.cuh")]:
         h.update(os.path.basename(f).encode())
         with open(f, "rb") as fh:
             h.update(fh.read())
