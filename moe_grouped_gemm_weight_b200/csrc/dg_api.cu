@@ -259,8 +259,12 @@ dg_status check_sizes(int mode, int rows, int N, int K, int G) {
 
 // Few-row problems (dense M <= 128, masked M_max <= 256) go to the swap-AB
 // split-K kernel: TN activation rows per tile (the smallest of 32/64/128 that
-// holds them), 128 weight rows per tile, and as many K splits (cluster size,
-// at most 8 and at most K/128) as keep two CTAs on every SM busy.
+// holds them), 128 weight rows per tile, and as many K splits (cluster size)
+// as keep two CTAs on every SM busy, with at most kSmallMaxSplit (4) slices
+// of at least kSmallMinSliceKb (8) K blocks each.  Per K block one CTA's
+// loop costs a fixed few hundred cycles (barrier hand-offs, MMA issue, the
+// promotion's TMEM round trips) that no deeper operand ring hides, so short
+// slices lose to their set-up and reduction.
 bool use_small(int mode, int rows) { return (mode == 0 && rows <= 128) || (mode == 2 && rows <= 256); }
 
 int small_tn(int mode, int rows) {
@@ -293,8 +297,11 @@ dg_status plan(int mode, int rows, int N, int K, int G, int num_sms, dg_plan* ou
         if (mode == 2 && expected_m > 0) active_m = G * cdiv(expected_m < rows ? expected_m : rows, tn);
         const long units = static_cast<long>(active_m) * n_blocks;
         int split = static_cast<int>((2L * num_sms) / (units > 0 ? units : 1));
-        const int max_split = dg::kSmallMaxSplit < K / dg::kBK ? dg::kSmallMaxSplit : K / dg::kBK;
-        split = split < 1 ? 1 : (split > max_split ? max_split : split);
+        constexpr int kSmallMinSliceKb = 8;
+        const int slices = K / dg::kBK / kSmallMinSliceKb;
+        const int max_split = dg::kSmallMaxSplit < slices ? dg::kSmallMaxSplit : slices;
+        if (split > max_split) split = max_split;
+        if (split < 1) split = 1;
         out->block_m = tn;
         out->block_n = 128;
         out->stages = small_stages(tn);

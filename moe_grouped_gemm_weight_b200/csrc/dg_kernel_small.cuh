@@ -28,7 +28,11 @@ constexpr int kSmallFirstEpiWarp = 4;
 constexpr int kSmallEpiWarps = 4;
 constexpr int kSmallScaleSlots = 16;
 constexpr int kSmallTmemCols = 256;
-constexpr int kSmallMaxSplit = 8;  // portable cluster size
+// Largest cluster (K splits per tile).  Measured on the M = 64 / 128 shapes of
+// the dense sweep, clusters of 6 and 8 CTAs were never faster than 4: at two
+// CTAs per SM an 8-CTA cluster lands on four SMs, and per slice the set-up and
+// the DSMEM reduction cost more than the shorter K loop saves.
+constexpr int kSmallMaxSplit = 4;
 
 template <int TN>
 struct SmallCfg {
@@ -36,7 +40,7 @@ struct SmallCfg {
     static constexpr int kTileBBytes = 128 * kBK;   // 128 weight rows
     static constexpr int kTileABytes = TN * kBK;    // TN activation rows
     static constexpr int kStageBytes = kTileBBytes + kTileABytes;
-    static constexpr int kStages = (96 * 1024) / kStageBytes;  // 5, 4 or 3 stages: ~96 KiB of ring
+    static constexpr int kStages = (96 * 1024) / kStageBytes;  // 4, 4 or 3 stages: ~96 KiB of ring
     static constexpr int kNBuf = kSmallTmemCols / TN > 4 ? 4 : kSmallTmemCols / TN;
     static constexpr int kChunks = TN / 32;
     static constexpr int kBatch = TN == 128 ? 1 : (kChunks < 2 ? kChunks : 2);

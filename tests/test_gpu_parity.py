@@ -266,12 +266,14 @@ def test_masked_under_cuda_graph_follows_device_counts(dgm):
 @pytest.mark.parametrize("M", [1, 17, 32, 33, 64, 100, 128])
 @pytest.mark.parametrize("sms", [148, 16, 3])
 def test_few_rows_split_k_variants(dgm, M, sms):
-    N, K = 520, 1536
+    # 35 K blocks: 4 slices of 8-9 blocks on 148 and 16 SMs, one on 3 SMs.
+    N, K = 520, 4480
     c = wl.dense_case(M, N, K, seed=M * 3 + sms)
     try:
         dgm.dg_set_num_sms(sms)
         plan = dgm.dg_make_plan(0, M, N, K, 1, sms)
         assert plan["swap_ab"] == 1
+        assert plan["split_k"] == (1 if sms == 3 else 4)
         got = run_dense(dgm, c)
     finally:
         dgm.dg_set_num_sms(0)
@@ -279,14 +281,25 @@ def test_few_rows_split_k_variants(dgm, M, sms):
     assert_close(got, ref, mag, f"few rows M={M} split={plan['split_k']}")
 
 
+@pytest.mark.parametrize("K,split", [(1024, 1), (2048, 2), (3072, 3), (3968, 3)])
+def test_few_rows_split_count_follows_k(dgm, K, split):
+    # Slices keep at least 8 K blocks: 8, 16, 24 and 31 blocks give 1, 2, 3
+    # and 3 slices (31 = 10 + 10 + 11).
+    c = wl.dense_case(64, 2112, K, seed=K)
+    assert dgm.dg_make_plan(0, 64, 2112, K, 1, 148)["split_k"] == split
+    got = run_dense(dgm, c)
+    ref, mag = oracle_dense(c)
+    assert_close(got, ref, mag, f"few rows K={K} split={split}")
+
+
 def test_few_rows_k_split_uneven(dgm):
-    # 7 K blocks over a cluster of up to 8 CTAs: some CTAs own one block, the
-    # split sizes differ, and the fixed-order sum must still match.
-    c = wl.dense_case(64, 2112, 896, seed=21)
+    # 35 K blocks over a cluster of 4 CTAs: slices of 8 and 9 blocks, and the
+    # fixed-order sum must still match.
+    c = wl.dense_case(64, 2112, 4480, seed=21)
     got = run_dense(dgm, c)
     ref, mag = oracle_dense(c)
     assert_close(got, ref, mag, "uneven split")
-    assert dgm.dg_make_plan(0, 64, 2112, 896, 1, 148)["split_k"] == 7
+    assert dgm.dg_make_plan(0, 64, 2112, 4480, 1, 148)["split_k"] == 4
 
 
 # ------------------------------------------- CTA-pair kernel (opt-in path) --

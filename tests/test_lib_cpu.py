@@ -90,7 +90,7 @@ def test_plan_is_consistent(mode, rows, N, K, G):
         # per tile, two CTAs per SM.
         assert rows <= (256 if mode == 2 else 128)
         assert p["block_n"] == 128 and p["block_m"] in (32, 64, 128)
-        assert 1 <= p["split_k"] <= min(8, K // 128)
+        assert 1 <= p["split_k"] <= max(1, min(4, K // 128 // 8))
         assert p["grid"] == p["tiles"] * p["split_k"]
         assert p["smem_bytes"] <= 113 * 1024
     else:
@@ -104,8 +104,9 @@ def test_plan_is_consistent(mode, rows, N, K, G):
 def test_few_row_plan_tile_and_split(M, tn):
     p = dg.dg_make_plan(0, M, 2112, 7168, 1, 148)
     assert p["swap_ab"] == 1 and p["block_m"] == tn
-    # 17 weight tiles; as many K splits as keep two CTAs per SM busy, at most 8.
-    assert p["n_blocks"] == 17 and p["split_k"] == min(8, (2 * 148) // 17)
+    # 17 weight tiles; as many K splits as keep two CTAs per SM busy, at most
+    # 4, each of at least 8 K blocks (56 here).
+    assert p["n_blocks"] == 17 and p["split_k"] == min(4, (2 * 148) // 17, 56 // 8)
     assert dg.dg_make_plan(0, 129, 2112, 7168, 1, 148)["swap_ab"] == 0
 
 
