@@ -42,8 +42,13 @@ constexpr int kFirstEpiWarp = 4;         // warps 4..11: promotion/epilogue
 constexpr int kEpiWarps = 8;
 constexpr int kTileABytes = kBM * kBK;   // 16 KiB of e4m3
 constexpr int kMaxMaskedGroups = 1024;   // masked mode: prefix table in smem
-constexpr int kScaleSlots = 16;          // depth of the scale ring
+constexpr int kScaleSlots = 16;          // depth of the scale ring, in K blocks
 constexpr int kScaleSlotFloats = kBM + 4;  // sa for 128 rows + up to 4 sb values
+// fp8_gemm_kernel fills and releases the scale ring kScaleGroup K blocks at a
+// time: its promotion waits on a scale barrier once per group instead of once
+// per K block.
+constexpr int kScaleGroup = 4;
+constexpr int kScaleGroups = kScaleSlots / kScaleGroup;
 constexpr int kStageOutBytes = 32 * 32 * 2;  // per promotion warp: 32 rows x 32 bf16 columns
 
 struct Params {
@@ -410,10 +415,12 @@ fp8_gemm_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtens
     } else if (warp == 2) {
         // ------------------------------------------------ scale producer ----
         // Per K block: lane l copies sa rows m0+4l..m0+4l+3 (16 bytes) and
-        // lanes 0..3 the tile's sb values; the copies run asynchronously and
-        // complete the slot's barrier when they land, so this warp only ever
-        // waits for a free slot.  Rows past the data and sb blocks past N are
-        // zero-filled, nothing outside the tensors is read.
+        // lanes 0..3 the tile's sb values; the copies run asynchronously.  A
+        // group of up to kScaleGroup consecutive K blocks of the tile shares
+        // one ring slot and one barrier, completed when all of its copies
+        // land, so this warp only ever waits for a free slot.  Rows past the
+        // data and sb blocks past N are zero-filled, nothing outside the
+        // tensors is read.
         int slot = 0;
         uint32_t sphase = 0;
         const int row_limit = p.M;  // rows of sa that exist (dense M, M_total or M_max)
@@ -430,16 +437,20 @@ fp8_gemm_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtens
             const int left = row_limit - r4;
             const uint32_t sa_bytes = left >= 4 ? 16u : (left > 0 ? static_cast<uint32_t>(left) * 4u : 0u);
             bool ok = true;
-            for (int kb = w.kb0; kb < w.kb1; ++kb) {
+            for (int kg = w.kb0; kg < w.kb1; kg += kScaleGroup) {
                 if (!mbar_wait(sempty + slot, sphase ^ 1u, abort_flag)) { ok = false; break; }
-                const uint32_t dst = smem_u32(sring + slot * kScaleSlotFloats);
-                const float* src = sa_bytes ? sa_base + static_cast<int64_t>(kb) * p.sa_stride + r4 : p.sa;
-                cp_async_16(dst + lane * 16, src, sa_bytes);
-                if (lane < 4)
-                    cp_async_4(dst + (kBM + lane) * 4, nb_ok ? sb_g + static_cast<int64_t>(nb) * nkb + kb : p.sb,
-                               nb_ok ? 4u : 0u);
+                const int n = min(kScaleGroup, w.kb1 - kg);
+                for (int j = 0; j < n; ++j) {
+                    const int kb = kg + j;
+                    const uint32_t dst = smem_u32(sring + (slot * kScaleGroup + j) * kScaleSlotFloats);
+                    const float* src = sa_bytes ? sa_base + static_cast<int64_t>(kb) * p.sa_stride + r4 : p.sa;
+                    cp_async_16(dst + lane * 16, src, sa_bytes);
+                    if (lane < 4)
+                        cp_async_4(dst + (kBM + lane) * 4, nb_ok ? sb_g + static_cast<int64_t>(nb) * nkb + kb : p.sb,
+                                   nb_ok ? 4u : 0u);
+                }
                 cp_async_arrive(sfull + slot);
-                if (++slot == kScaleSlots) { slot = 0; sphase ^= 1u; }
+                if (++slot == kScaleGroups) { slot = 0; sphase ^= 1u; }
             }
             if (!ok) break;
         }
@@ -494,8 +505,9 @@ fp8_gemm_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtens
             for (int j = 0; j < C::kColsPerWarp / 2; ++j) acc[j] = make_float2(0.f, 0.f);
 
             for (int kb = w.kb0; kb < w.kb1; ++kb) {
-                if (!mbar_wait(sfull + slot, sphase, abort_flag)) { ok = false; break; }
-                const float* sc = sring + slot * kScaleSlotFloats;
+                const int jg = (kb - w.kb0) % kScaleGroup;  // K block inside its scale group
+                if (jg == 0 && !mbar_wait(sfull + slot, sphase, abort_flag)) { ok = false; break; }
+                const float* sc = sring + (slot * kScaleGroup + jg) * kScaleSlotFloats;
                 const float s_a = sc[r];
                 float2 s2[C::kChunks];
 #pragma unroll
@@ -503,9 +515,12 @@ fp8_gemm_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtens
                     const float s = s_a * sc[kBM + sb_sel[c]];
                     s2[c] = make_float2(s, s);
                 }
-                __syncwarp();
-                if (lane == 0) mbar_arrive(sempty + slot);
-                if (++slot == kScaleSlots) { slot = 0; sphase ^= 1u; }
+                if (jg == kScaleGroup - 1 || kb == w.kb1 - 1) {
+                    // The group's last K block has read its scales: release the slot.
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(sempty + slot);
+                    if (++slot == kScaleGroups) { slot = 0; sphase ^= 1u; }
+                }
 
                 if (!mbar_wait(tfull + buf, bphase, abort_flag)) { ok = false; break; }
                 tc_fence_after();
