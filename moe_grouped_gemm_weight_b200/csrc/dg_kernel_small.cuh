@@ -26,7 +26,11 @@ namespace dg {
 constexpr int kSmallThreads = 256;
 constexpr int kSmallFirstEpiWarp = 4;
 constexpr int kSmallEpiWarps = 4;
-constexpr int kSmallScaleSlots = 16;
+constexpr int kSmallScaleSlots = 16;  // depth of the scale ring, in K blocks
+// The scale ring is filled and released kSmallScaleGroup K blocks at a time,
+// so the promotion waits on a scale barrier once per group.
+constexpr int kSmallScaleGroup = 4;
+constexpr int kSmallScaleGroups = kSmallScaleSlots / kSmallScaleGroup;
 constexpr int kSmallTmemCols = 256;
 // Largest cluster (K splits per tile).  Measured on the M = 64 / 128 shapes of
 // the dense sweep, clusters of 6 and 8 CTAs were never faster than 4: at two
@@ -213,9 +217,10 @@ fp8_gemm_swapab_kernel(const __grid_constant__ Params p, const __grid_constant__
         } else if (warp == 2) {
             // ------------------------------------------- scale producer ----
             // Per K block: sa[m0 .. m0+TN) (lane l copies TN/32 consecutive
-            // rows) and sb[n0/128] (lane 0), copied asynchronously; the copies
-            // complete the slot's barrier when they land.  Rows past the data
-            // are zero-filled and never read.
+            // rows) and sb[n0/128] (lane 0), copied asynchronously.  Up to
+            // kSmallScaleGroup consecutive K blocks share a ring slot whose
+            // barrier completes when all of their copies land.  Rows past the
+            // data are zero-filled and never read.
             constexpr int kPer = TN / 32;  // floats per lane
             const float* sa_base = p.sa + (MODE == kMasked ? static_cast<int64_t>(g) * nkb * p.sa_stride : 0);
             const float* sb_row = p.sb + (static_cast<int64_t>(g) * p.nbn + n0 / 128) * nkb;
@@ -224,19 +229,23 @@ fp8_gemm_swapab_kernel(const __grid_constant__ Params p, const __grid_constant__
             const uint32_t sa_bytes = left >= kPer ? 4u * kPer : (left > 0 ? 4u * static_cast<uint32_t>(left) : 0u);
             int slot = 0;
             uint32_t sphase = 0;
-            for (int kb = kb0; kb < kb1; ++kb) {
+            for (int kg = kb0; kg < kb1; kg += kSmallScaleGroup) {
                 if (!mbar_wait(sempty + slot, sphase ^ 1u, abort_flag)) break;
-                const uint32_t dst = smem_u32(sring + slot * (TN + 4));
-                const float* src = sa_bytes ? sa_base + static_cast<int64_t>(kb) * p.sa_stride + r : p.sa;
-                if (kPer == 4)
-                    cp_async_16(dst + lane * 16, src, sa_bytes);
-                else if (kPer == 2)
-                    cp_async_8(dst + lane * 8, src, sa_bytes);
-                else
-                    cp_async_4(dst + lane * 4, src, sa_bytes);
-                if (lane == 0) cp_async_4(dst + TN * 4, sb_row + kb, 4u);
+                const int n = min(kSmallScaleGroup, kb1 - kg);
+                for (int j = 0; j < n; ++j) {
+                    const int kb = kg + j;
+                    const uint32_t dst = smem_u32(sring + (slot * kSmallScaleGroup + j) * (TN + 4));
+                    const float* src = sa_bytes ? sa_base + static_cast<int64_t>(kb) * p.sa_stride + r : p.sa;
+                    if (kPer == 4)
+                        cp_async_16(dst + lane * 16, src, sa_bytes);
+                    else if (kPer == 2)
+                        cp_async_8(dst + lane * 8, src, sa_bytes);
+                    else
+                        cp_async_4(dst + lane * 4, src, sa_bytes);
+                    if (lane == 0) cp_async_4(dst + TN * 4, sb_row + kb, 4u);
+                }
                 cp_async_arrive(sfull + slot);
-                if (++slot == kSmallScaleSlots) { slot = 0; sphase ^= 1u; }
+                if (++slot == kSmallScaleGroups) { slot = 0; sphase ^= 1u; }
             }
             asm volatile("cp.async.wait_all;" ::: "memory");
         }
@@ -251,11 +260,12 @@ fp8_gemm_swapab_kernel(const __grid_constant__ Params p, const __grid_constant__
         int buf = 0, slot = 0;
         uint32_t bphase = 0, sphase = 0;
         for (int kb = kb0; kb < kb1; ++kb) {
-            if (!mbar_wait(sfull + slot, sphase, abort_flag)) break;
+            const int jg = (kb - kb0) % kSmallScaleGroup;  // K block inside its scale group
+            if (jg == 0 && !mbar_wait(sfull + slot, sphase, abort_flag)) break;
             if (!mbar_wait(tfull + buf, bphase, abort_flag)) break;
             tc_fence_after();
             // Scales of this K block: s[j] = sa[m0 + j] * sb, formed here.
-            const float* slot_f = sring + slot * (TN + 4);
+            const float* slot_f = sring + (slot * kSmallScaleGroup + jg) * (TN + 4);
             const float2* sc = reinterpret_cast<const float2*>(slot_f);
             const float s_b = slot_f[TN];
             const float2 sb2 = make_float2(s_b, s_b);
@@ -282,9 +292,12 @@ fp8_gemm_swapab_kernel(const __grid_constant__ Params p, const __grid_constant__
                         acc[q] = __ffma2_rn(pv, __fmul2_rn(sc[q], sb2), acc[q]);
                     }
             }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(sempty + slot);
-            if (++slot == kSmallScaleSlots) { slot = 0; sphase ^= 1u; }
+            if (jg == kSmallScaleGroup - 1 || kb == kb1 - 1) {
+                // The group's last K block is done with its scales: release the slot.
+                __syncwarp();
+                if (lane == 0) mbar_arrive(sempty + slot);
+                if (++slot == kSmallScaleGroups) { slot = 0; sphase ^= 1u; }
+            }
             if (++buf == kNBuf) { buf = 0; bphase ^= 1u; }
         }
         // The ring is idle once this CTA's last partial has been read out of
