@@ -258,11 +258,10 @@ dg_status check_sizes(int mode, int rows, int N, int K, int G) {
 }
 
 // Few-row problems (dense M <= 128, masked M_max <= 256) go to the swap-AB
-// split-K kernel: TN activation rows per tile (the smallest of 32/64/128 that
-// holds them), 128 weight rows per tile, and as many K splits (cluster size)
-// as keep two CTAs on every SM busy, with at most kSmallMaxSplit (4) slices
-// of at least kSmallMinSliceKb (8) K blocks each.  Per K block one CTA's
-// loop costs a fixed few hundred cycles (barrier hand-offs, MMA issue, the
+// split-K kernel: TN activation rows per tile (masked: the smallest of
+// 32/64/128 that holds them; dense: see small_dense_tn), 128 weight rows per
+// tile, and K split over a cluster (small_split).  Per K block one CTA's loop
+// costs a fixed few hundred cycles (barrier hand-offs, MMA issue, the
 // promotion's TMEM round trips) that no deeper operand ring hides, so short
 // slices lose to their set-up and reduction.
 bool use_small(int mode, int rows) { return (mode == 0 && rows <= 128) || (mode == 2 && rows <= 256); }
@@ -270,6 +269,37 @@ bool use_small(int mode, int rows) { return (mode == 0 && rows <= 128) || (mode 
 int small_tn(int mode, int rows) {
     const int t = mode == 2 ? (rows < 128 ? rows : 128) : rows;
     return t <= 32 ? 32 : t <= 64 ? 64 : 128;
+}
+
+// K splits for `units` few-row tiles: as many as keep two CTAs on every SM
+// busy, at most kSmallMaxSplit slices of at least kSmallMinSliceKb K blocks.
+int small_split(long units, int nkb, int num_sms) {
+    constexpr int kSmallMinSliceKb = 8;
+    int split = static_cast<int>((2L * num_sms) / (units > 0 ? units : 1));
+    const int slices = nkb / kSmallMinSliceKb;
+    if (split > dg::kSmallMaxSplit) split = dg::kSmallMaxSplit;
+    if (split > slices) split = slices;
+    return split < 1 ? 1 : split;
+}
+
+// Dense few-row calls may cut the activation rows into smaller tiles (TN / 2,
+// TN / 4, at least 32): more tiles, more CTAs in flight.  Per K block one
+// CTA's loop costs a roughly fixed time that grows with TN (measured with
+// clock stamps: about 0.44 / 0.56 / 0.75 us for TN = 32 / 64 / 128), so the
+// estimate is waves x K blocks per CTA x that cost; ties keep the larger TN.
+int small_dense_tn(int rows, int N, int nkb, int num_sms) {
+    const int tn0 = small_tn(0, rows);
+    int best_tn = tn0;
+    long best = -1;
+    for (int tn = tn0; tn >= 32; tn /= 2) {
+        const long units = static_cast<long>(cdiv(rows, tn)) * cdiv(N, 128);
+        const int split = small_split(units, nkb, num_sms);
+        const long waves = (units * split + 2L * num_sms - 1) / (2L * num_sms);
+        const long per_kb = tn == 32 ? 44 : tn == 64 ? 56 : 75;
+        const long cost = waves * ((nkb + split - 1) / split) * per_kb;
+        if (best < 0 || cost < best) { best = cost; best_tn = tn; }
+    }
+    return best_tn;
 }
 
 int small_smem(int tn) {
@@ -287,7 +317,7 @@ dg_status plan(int mode, int rows, int N, int K, int G, int num_sms, dg_plan* ou
     if (num_sms <= 0) return fail(DG_ERR_INVALID_ARG, "num_sms must be positive");
     *out = dg_plan{};
     if (layout == 0 && use_small(mode, rows)) {
-        const int tn = small_tn(mode, rows);
+        const int tn = mode == 0 ? small_dense_tn(rows, N, K / dg::kBK, num_sms) : small_tn(mode, rows);
         const int per_group = cdiv(rows, tn);
         const int m_blocks = mode == 2 ? G * per_group : per_group;
         const int n_blocks = cdiv(N, 128);
@@ -296,12 +326,7 @@ dg_status plan(int mode, int rows, int N, int K, int G, int num_sms, dg_plan* ou
         int active_m = m_blocks;
         if (mode == 2 && expected_m > 0) active_m = G * cdiv(expected_m < rows ? expected_m : rows, tn);
         const long units = static_cast<long>(active_m) * n_blocks;
-        int split = static_cast<int>((2L * num_sms) / (units > 0 ? units : 1));
-        constexpr int kSmallMinSliceKb = 8;
-        const int slices = K / dg::kBK / kSmallMinSliceKb;
-        const int max_split = dg::kSmallMaxSplit < slices ? dg::kSmallMaxSplit : slices;
-        if (split > max_split) split = max_split;
-        if (split < 1) split = 1;
+        const int split = small_split(units, K / dg::kBK, num_sms);
         out->block_m = tn;
         out->block_n = 128;
         out->stages = small_stages(tn);

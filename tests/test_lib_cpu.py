@@ -100,14 +100,25 @@ def test_plan_is_consistent(mode, rows, N, K, G):
         assert p["smem_bytes"] <= 227 * 1024
 
 
-@pytest.mark.parametrize("M,tn", [(1, 32), (32, 32), (33, 64), (64, 64), (65, 128), (128, 128)])
-def test_few_row_plan_tile_and_split(M, tn):
-    p = dg.dg_make_plan(0, M, 2112, 7168, 1, 148)
-    assert p["swap_ab"] == 1 and p["block_m"] == tn
-    # 17 weight tiles; as many K splits as keep two CTAs per SM busy, at most
-    # 4, each of at least 8 K blocks (56 here).
-    assert p["n_blocks"] == 17 and p["split_k"] == min(4, (2 * 148) // 17, 56 // 8)
-    assert dg.dg_make_plan(0, 129, 2112, 7168, 1, 148)["swap_ab"] == 0
+@pytest.mark.parametrize("M,N,K,tn,split", [
+    (1, 2112, 7168, 32, 4), (32, 2112, 7168, 32, 4),
+    # dense tiles of fewer rows than the call has, where more CTAs pay off
+    (64, 2112, 7168, 32, 4), (128, 2112, 7168, 32, 4), (128, 4096, 7168, 64, 4), (128, 7168, 2048, 64, 2),
+    # enough weight tiles already: the smallest TN that holds the rows
+    (64, 24576, 1536, 64, 1), (128, 24576, 1536, 128, 1), (128, 32768, 512, 128, 1), (128, 7168, 16384, 128, 4),
+])
+def test_few_row_plan_tile_and_split(M, N, K, tn, split):
+    p = dg.dg_make_plan(0, M, N, K, 1, 148)
+    assert p["swap_ab"] == 1 and p["block_m"] == tn and p["split_k"] == split
+    assert p["m_blocks"] == -(-M // tn) and p["n_blocks"] == -(-N // 128)
+    assert dg.dg_make_plan(0, 129, N, K, 1, 148)["swap_ab"] == 0
+
+
+def test_few_row_plan_never_exceeds_the_rows_tile():
+    for M in range(1, 129):
+        p = dg.dg_make_plan(0, M, 520, 4480, 1, 148)
+        assert p["block_m"] <= (32 if M <= 32 else 64 if M <= 64 else 128)
+        assert 1 <= p["split_k"] <= 4 and p["grid"] == p["tiles"] * p["split_k"]
 
 
 @pytest.mark.parametrize("args,expect", [
