@@ -337,6 +337,8 @@ dg_status plan(int mode, int rows, int N, int K, int G, int num_sms, dg_plan* ou
         out->smem_bytes = small_smem(tn);
         out->swap_ab = 1;
         out->split_k = split;
+        out->cta_pair = 0;
+        out->tail_split = 1;  // the cluster split replaces the tail split
         return DG_OK;
     }
     const int m_blocks = (mode == 2) ? G * cdiv(rows, dg::kBM) : cdiv(rows, dg::kBM);
@@ -363,6 +365,7 @@ dg_status plan(int mode, int rows, int N, int K, int G, int num_sms, dg_plan* ou
         out->swap_ab = 0;
         out->split_k = 1;
         out->cta_pair = 1;
+        out->tail_split = 1;  // pair tiles have no K-split tail
         return DG_OK;
     }
     out->block_m = dg::kBM;
