@@ -25,6 +25,9 @@ MUTANTS = {
     "products_lose_sign": ("p += t;", "p += fabs(t);"),
     "contiguous_ignores_group": ("B + (int64_t)g * N * K, sb + (int64_t)g * nbn * nkb, N, K,\n                 D + m * N",
                                  "B, sb, N, K,\n                 D + m * N"),
+    "mag_unscaled": ("acc_mag += fabs(s) * pmag;", "acc_mag += pmag;"),
+    "mag_doubled": ("acc_mag += fabs(s) * pmag;", "acc_mag += 2.0 * fabs(s) * pmag;"),
+    "mag_signed_products": ("pmag += fabs(t);", "pmag += t;"),
     "masked_off_by_one": ("if (m >= masked_m[g]) continue;", "if (m > masked_m[g]) continue;"),
     "cast_ties_away": ("if (rem > 0.5 || (rem == 0.5 && fmod(f, 2.0) == 1.0)) f += 1.0;", "if (rem >= 0.5) f += 1.0;"),
     "cast_sign_lost": ("const uint8_t sign = signbit(x) ? 0x80 : 0x00;", "const uint8_t sign = 0x00;"),

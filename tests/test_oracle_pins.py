@@ -29,8 +29,12 @@ def dequant_torch(codes) -> np.ndarray:
     return t.to(torch.float64).numpy()
 
 
-def brute_force(case: wl.Case, g: int = 0, rows=None) -> np.ndarray:
-    """D64 by dequantising A and B (with their scales) to float64 and one matmul."""
+def brute_force(case: wl.Case, g: int = 0, rows=None, with_mag: bool = False):
+    """D64 by dequantising A and B (with their scales) to float64 and one matmul.
+
+    With ``with_mag`` it also returns |A_s| @ |B_s|^T, the sum over k of the
+    magnitudes of the scaled products: the tolerance term the oracle reports
+    as MAG, computed here from the dequantised operands instead of per block."""
     K, N = case.K, case.N
     nkb = case.nkb
     A = case.A.numpy().reshape(-1, K)
@@ -47,7 +51,14 @@ def brute_force(case: wl.Case, g: int = 0, rows=None) -> np.ndarray:
     sb = case.sb.numpy().reshape(-1, case.nbn, nkb)[g].astype(np.float64)
     nblk = np.arange(N) // 128
     B_s = dequant_torch(B) * sb[nblk][:, kblk]
+    if with_mag:
+        return A_s @ B_s.T, np.abs(A_s) @ np.abs(B_s).T
     return A_s @ B_s.T
+
+
+def assert_mag_matches(mag, mag_ref):
+    """MAG is a sum of non-negative terms in another order: equal to 1e-12 relative."""
+    assert np.all(np.abs(mag - mag_ref) <= 1e-12 * mag_ref), "MAG differs from |A_s| @ |B_s|^T"
 
 
 def run_dense(case: wl.Case, **kw):
@@ -159,7 +170,11 @@ BRUTE_SHAPES = [(3, 5, 2), (1, 128, 1), (2, 256, 3), (5, 384, 129), (65, 257, 13
 def test_dense_matches_bruteforce_dequantised_matmul(M, K, N, stress):
     case = wl.dense_case(M, N, K, seed=11 + M + K + N, stress=stress)
     D, D64, MAG = run_dense(case)
-    ref = brute_force(case)
+    ref, mag_ref = brute_force(case, with_mag=True)
+    # MAG must be the scaled magnitude sum itself, pinned from both sides:
+    # a MAG that lost its scales or a factor would make every tolerance
+    # built on it wrong.
+    assert_mag_matches(MAG, mag_ref)
     # Two FP64 summation orders differ by at most ~K*eps*sum|terms|.
     assert np.all(np.abs(D64 - ref) <= 1e-12 * MAG)
     assert_bf16_of(D, ref, rel=1e-9)
@@ -309,7 +324,8 @@ def test_contiguous_equals_dense_per_segment_and_leaves_padding():
         rows = np.nonzero(idx == g)[0]
         if rows.size == 0:
             continue
-        ref = brute_force(case, g=g, rows=rows)
+        ref, mag_ref = brute_force(case, g=g, rows=rows, with_mag=True)
+        assert_mag_matches(MAG[rows], mag_ref)
         assert np.all(np.abs(D64[rows] - ref) <= 1e-12 * MAG[rows])
         assert_bf16_of(D[rows], ref, rel=1e-9)
 
@@ -332,7 +348,8 @@ def test_masked_equals_dense_on_valid_rows_and_leaves_the_rest():
     for g, mm in enumerate([0, 70, 33]):
         assert np.all(D[g, mm:] == SENT)
         if mm:
-            ref = brute_force(case, g=g, rows=np.arange(mm))
+            ref, mag_ref = brute_force(case, g=g, rows=np.arange(mm), with_mag=True)
+            assert_mag_matches(MAG[g, :mm], mag_ref)
             assert np.all(np.abs(D64[g, :mm] - ref) <= 1e-12 * MAG[g, :mm])
             assert_bf16_of(D[g, :mm], ref, rel=1e-9)
 
