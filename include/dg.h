@@ -20,12 +20,18 @@
  *             keeps them past the call.
  *  Workspace  Dense calls whose last wave of tiles is partial split those
  *             tiles along K; the slices' FP32 partials go to a workspace the
- *             library allocates ONCE per (device, stream) on first need (one
- *             128 x BN FP32 tile per SM, about 19 MB on a B200, zeroed) and
- *             keeps until exit.  While a stream is being captured into a CUDA
+ *             library allocates once per (device, stream) on first need (one
+ *             128 x BN FP32 tile per SM, about 19 MB on a B200, zeroed).  At
+ *             most four streams per device hold one: the first split call on
+ *             a fifth stream frees the least recently used workspace (its
+ *             cudaFree waits for the device), so short-lived streams do not
+ *             accumulate memory.  While a stream is being captured into a CUDA
  *             graph and has no workspace yet, calls do not split (results are
  *             the same up to FP32 summation order); make one call on the
- *             stream before capturing to keep the split.
+ *             stream before capturing to keep the split, and capture on at
+ *             most four streams per device that way.  dg_get_device_error()
+ *             clears the workspaces' ready flags when it reports
+ *             DG_DEVERR_TIMEOUT, so a timed-out launch leaves none set.
  *  Layouts    A   uint8 (e4m3 codes) [rows][K], K contiguous.
  *             B   uint8 (e4m3 codes) [G][N][K], K contiguous ("NT": the RHS is
  *                 stored transposed).  G = 1 for the dense call.
@@ -159,6 +165,13 @@ DG_API dg_status dg_k_grouped_fp8_gemm_tn(uint16_t* D, const uint8_t* A, const f
  */
 DG_API dg_status dg_fp8_gemm_nt_ue8m0(uint16_t* D, const uint8_t* A, const float* sa, int sa_stride,
                                       const uint8_t* B, const float* sb, int M, int N, int K, void* stream);
+
+/*
+ * Number of K-split workspaces (see "Workspace" above) the library holds,
+ * over all devices and streams.  Host-only, no synchronisation; for tests and
+ * memory accounting.
+ */
+DG_API int dg_get_workspace_count(void);
 
 /*
  * Dense GEMM that allocates nothing.  The pages describe no such call; it

@@ -88,6 +88,8 @@ def lib() -> ctypes.CDLL:
             L.dg_get_tma_aligned_size.argtypes = [I, I]
             L.dg_get_device_error.restype = I
             L.dg_get_device_error.argtypes = [ctypes.POINTER(I)]
+            L.dg_get_workspace_count.restype = I
+            L.dg_get_workspace_count.argtypes = []
             L.dg_status_string.restype = ctypes.c_char_p
             L.dg_status_string.argtypes = [I]
             L.dg_last_error_message.restype = ctypes.c_char_p
@@ -240,6 +242,10 @@ def dg_get_device_error() -> int:
     code = ctypes.c_int(0)
     _check("dg_get_device_error", lib().dg_get_device_error(ctypes.byref(code)))
     return int(code.value)
+
+
+def dg_get_workspace_count() -> int:
+    return int(lib().dg_get_workspace_count())
 
 
 def dg_make_plan(mode: int, rows: int, N: int, K: int, G: int, num_sms: int) -> dict:

@@ -2,7 +2,8 @@
 // validation, the launch plan (tile shape, ring depth, grid), TMA tensor-map
 // encoding and kernel dispatch.  Nothing here reads device memory or
 // synchronises, except dg_get_device_error(); the only device allocation is
-// the per-(device, stream) K-split workspace, made once on first need.
+// the per-(device, stream) K-split workspace, made on first need (at most four
+// streams per device keep one).
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -627,26 +628,47 @@ int choose_raster(int m_blocks, int n_blocks, int block_m, int block_n, int K, i
     return best;
 }
 
-// Workspace for the K-split tail: per (device, stream), allocated once on
-// first need, never during stream capture.  Holds one 128 x 256 FP32 partial
-// per SM (the split keeps fewer than grid <= SMs partials) and their flags.
+// Workspace for the K-split tail: per (device, stream), allocated on first
+// need, never during stream capture.  Holds one 128 x 256 FP32 partial per SM
+// (the split keeps fewer than grid <= SMs partials) and their flags.  At most
+// kMaxTailWorkspaces streams per device keep one: the first call on a further
+// stream frees the least recently used (cudaFree waits for the whole device,
+// so no launch still uses it).  Allocation and freeing run in relaxed capture
+// mode, so that another thread's CUDA-graph capture is not invalidated; if
+// either fails the call runs without the split (same result up to FP32
+// summation order).
+constexpr int kMaxTailWorkspaces = 4;
+
 struct TailWorkspace {
     float* partials = nullptr;
     unsigned int* flags = nullptr;
+    size_t flag_bytes = 0;
+    uint64_t last_use = 0;
+};
+
+std::mutex g_ws_mu;
+std::map<std::pair<int, cudaStream_t>, TailWorkspace> g_ws;
+uint64_t g_ws_clock = 0;
+
+// Allocation / free helpers for the workspace: relaxed capture mode for the
+// calling thread, restored afterwards.
+struct RelaxedCapture {
+    cudaStreamCaptureMode prev = cudaStreamCaptureModeRelaxed;
+    RelaxedCapture() { cudaThreadExchangeStreamCaptureMode(&prev); }
+    ~RelaxedCapture() { cudaThreadExchangeStreamCaptureMode(&prev); }
 };
 
 bool tail_workspace(cudaStream_t stream, TailWorkspace* out) {
-    static std::mutex mu;
-    static std::map<std::pair<int, cudaStream_t>, TailWorkspace> spaces;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) {
         cudaGetLastError();
         return false;
     }
-    std::lock_guard<std::mutex> lock(mu);
+    std::lock_guard<std::mutex> lock(g_ws_mu);
     auto key = std::make_pair(dev, stream);
-    auto it = spaces.find(key);
-    if (it != spaces.end()) {
+    auto it = g_ws.find(key);
+    if (it != g_ws.end()) {
+        it->second.last_use = ++g_ws_clock;
         *out = it->second;
         return true;
     }
@@ -658,21 +680,57 @@ bool tail_workspace(cudaStream_t stream, TailWorkspace* out) {
     if (cs != cudaStreamCaptureStatusNone) return false;
     const int sms = device_sm_count();
     if (sms <= 0) return false;
+    RelaxedCapture relaxed;
+    int on_dev = 0;
+    auto lru = g_ws.end();
+    for (auto j = g_ws.begin(); j != g_ws.end(); ++j) {
+        if (j->first.first != dev) continue;
+        ++on_dev;
+        if (lru == g_ws.end() || j->second.last_use < lru->second.last_use) lru = j;
+    }
+    if (on_dev >= kMaxTailWorkspaces) {
+        if (cudaFree(lru->second.partials) != cudaSuccess || cudaFree(lru->second.flags) != cudaSuccess) {
+            cudaGetLastError();
+            return false;
+        }
+        g_ws.erase(lru);
+    }
     TailWorkspace ws;
     const size_t part_bytes = static_cast<size_t>(sms) * dg::kBM * 256 * sizeof(float);
-    const size_t flag_bytes = static_cast<size_t>(sms) * sizeof(unsigned int);
+    ws.flag_bytes = static_cast<size_t>(sms) * sizeof(unsigned int);
     if (cudaMalloc(&ws.partials, part_bytes) != cudaSuccess) {
         cudaGetLastError();
         return false;
     }
-    if (cudaMalloc(&ws.flags, flag_bytes) != cudaSuccess || cudaMemset(ws.flags, 0, flag_bytes) != cudaSuccess) {
+    if (cudaMalloc(&ws.flags, ws.flag_bytes) != cudaSuccess || cudaMemset(ws.flags, 0, ws.flag_bytes) != cudaSuccess) {
         cudaGetLastError();
         cudaFree(ws.partials);
         return false;
     }
-    spaces[key] = ws;
+    ws.last_use = ++g_ws_clock;
+    g_ws[key] = ws;
     *out = ws;
     return true;
+}
+
+// After a bounded wait ran out, a late slice may have raised a ready flag
+// that no launch consumes; clear every workspace flag on the current device
+// (the caller has synchronised it).
+void clear_workspace_flags() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        return;
+    }
+    std::lock_guard<std::mutex> lock(g_ws_mu);
+    for (auto& kv : g_ws)
+        if (kv.first.first == dev && cudaMemset(kv.second.flags, 0, kv.second.flag_bytes) != cudaSuccess)
+            cudaGetLastError();
+}
+
+int tail_workspace_count() {
+    std::lock_guard<std::mutex> lock(g_ws_mu);
+    return static_cast<int>(g_ws.size());
 }
 
 dg::Params make_params(uint16_t* D, const float* sa, int sa_stride, const float* sb, int rows, int N, int K, int G,
@@ -1121,6 +1179,8 @@ int dg_get_tma_aligned_size(int x, int elem_bytes) {
     return cdiv(x, per) * per;
 }
 
+int dg_get_workspace_count(void) { return tail_workspace_count(); }
+
 dg_status dg_get_device_error(int* code) {
     if (!code) return fail(DG_ERR_INVALID_ARG, "null code pointer");
     cudaError_t e = cudaDeviceSynchronize();
@@ -1129,6 +1189,7 @@ dg_status dg_get_device_error(int* code) {
     e = cudaMemcpyFromSymbol(&v, dg::g_dg_error, sizeof(v));
     if (e == cudaSuccess) e = cudaMemcpyToSymbol(dg::g_dg_error, &zero, sizeof(zero));
     if (e != cudaSuccess) return fail(DG_ERR_CUDA, "reading the device error word: %s", cudaGetErrorString(e));
+    if (v & DG_DEVERR_TIMEOUT) clear_workspace_flags();
     *code = static_cast<int>(v);
     return ok();
 }

@@ -360,6 +360,32 @@ def test_tail_split_matches_oracle_and_is_deterministic(dgm, M, N, K, sms, split
     assert dgm.dg_get_device_error() == 0
 
 
+def test_tail_split_workspaces_stay_bounded_over_many_streams(dgm):
+    # One split call on each of six fresh streams: at most four per device
+    # keep a workspace (the least recently used is freed), and every stream's
+    # result is the same bits as the default stream's.
+    M, N, K, sms = 384, 1792, 8192, 20
+    c = wl.dense_case(M, N, K, seed=77).to("cuda")
+    try:
+        dgm.dg_set_num_sms(sms)
+        assert dgm.dg_make_plan(0, M, N, K, 1, sms)["tail_split"] > 1
+        D0 = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+        dgm.dg_fp8_gemm_nt(D0, c.A, c.sa, c.sa_stride, c.B, c.sb)
+        torch.cuda.synchronize()
+        for i in range(6):
+            st = torch.cuda.Stream()
+            D = torch.zeros(M, N, dtype=torch.bfloat16, device="cuda")
+            torch.cuda.synchronize()
+            with torch.cuda.stream(st):
+                dgm.dg_fp8_gemm_nt(D, c.A, c.sa, c.sa_stride, c.B, c.sb)
+            st.synchronize()
+            assert torch.equal(D.view(torch.int16), D0.view(torch.int16)), f"stream {i}"
+            assert dgm.dg_get_workspace_count() <= 4
+    finally:
+        dgm.dg_set_num_sms(0)
+    assert dgm.dg_get_device_error() == 0
+
+
 # ------------------------------------- back-to-back launches (PDL) --------
 # With DG_PDL=1 GEMM launches allow programmatic dependent launch: a kernel may
 # start its set-up while the previous kernel in the stream finishes.  It must

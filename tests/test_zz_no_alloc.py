@@ -1,12 +1,17 @@
-"""GPU: the allocation-free dense entry point against the ordinary one.
+"""GPU: the allocation-free dense entry point against the oracle.
 
-dg_fp8_gemm_nt_noalloc keeps the K-split scratch in a static device array that
-every call shares, so each case runs it twice in a row, after other cases have
-left their partials and flags there, and compares both results with
-dg_fp8_gemm_nt's within the parity tolerance
+dg_fp8_gemm_nt_noalloc exists for callers that must not allocate device
+memory once running (a serving loop that reserved HBM for its own pool, code
+that cannot take the synchronisation cudaMalloc/cudaFree may bring): it keeps
+the K-split scratch in a static device array that every call shares.  Each case
+runs it twice in a row, after other cases have left their partials and flags
+there, and compares both results with the CPU oracle's D within the parity
+tolerance
     |D_new - D_ref| <= 2^-7 * |D_ref| + 1e-4 * MAG,   MAG = sum_k |sa*sb*a_k*b_k|
-(MAG from the oracle, on one row of every 128-row block plus the edges).
-Bytes around D are compared bit-exactly against a sentinel.
+on one row of every 128-row block plus the edges.  The ordinary entry point's
+result is compared the same way, and the cases that are meant to use the
+scratch are checked to plan a K split.  Bytes around D are compared
+bit-exactly against a sentinel.
 """
 import numpy as np
 import pytest
@@ -20,10 +25,11 @@ pytestmark = pytest.mark.gpu
 SENTINEL = 0x7FBF
 GUARD = 256
 
-# (M, N, K, SM cap or 0 for all): K-split tails of 3, 68 and 56 partials, a
-# ragged shape and a few-row shape that take no scratch, then the first again.
-CASES = [(384, 1792, 8192, 20), (4096, 4096, 7168, 0), (1000, 1000, 1024, 0), (64, 2112, 7168, 0),
-         (4096, 7168, 16384, 0), (384, 1792, 8192, 20)]
+# (M, N, K, SM cap or 0 for all, uses the scratch): K-split tails of 3, 68 and
+# 56 partials, a ragged shape and a few-row shape that take no scratch, then
+# the first again.
+CASES = [(384, 1792, 8192, 20, True), (4096, 4096, 7168, 0, True), (1000, 1000, 1024, 0, False),
+         (64, 2112, 7168, 0, False), (4096, 7168, 16384, 0, True), (384, 1792, 8192, 20, True)]
 
 
 @pytest.fixture(scope="module")
@@ -50,25 +56,29 @@ def _f64(bits):
     return (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
 
 
-def test_noalloc_matches_dense_entry_on_consecutive_calls(dgm):
-    for i, (M, N, K, sms) in enumerate(CASES):
+def test_noalloc_matches_oracle_on_consecutive_calls(dgm):
+    import torch as _t
+    sms_all = _t.cuda.get_device_properties(0).multi_processor_count
+    for i, (M, N, K, sms, split) in enumerate(CASES):
+        plan = dgm.dg_make_plan(0, M, N, K, 1, sms or sms_all)
+        assert (plan["tail_split"] > 1) == split, (M, N, K, sms, plan)
         c = wl.dense_case(M, N, K, seed=100 + i, device="cuda")
         try:
             dgm.dg_set_num_sms(sms)
-            ref = _call(dgm.dg_fp8_gemm_nt, c)
+            ref_entry = _call(dgm.dg_fp8_gemm_nt, c)
             first = _call(dgm.dg_fp8_gemm_nt_noalloc, c)
             second = _call(dgm.dg_fp8_gemm_nt_noalloc, c)
         finally:
             dgm.dg_set_num_sms(0)
         rows = np.array(sorted({0, M - 1} | set(range(min(M - 1, 77), M, 128))), dtype=np.int64)
         cc = c.to("cpu")
-        _, _, mag = oracle.gemm_nt(cc.A.numpy(), cc.sa.numpy(), cc.sa_stride, cc.B.numpy(), cc.sb.numpy(),
-                                   M, N, K, rows=rows, want_d64=False)
-        r = _f64(ref[rows])
+        d_bits, _, mag = oracle.gemm_nt(cc.A.numpy(), cc.sa.numpy(), cc.sa_stride, cc.B.numpy(), cc.sb.numpy(),
+                                        M, N, K, rows=rows, want_d64=False)
+        r = _f64(d_bits[rows])
         tol = 2.0 ** -7 * np.abs(r) + 1e-4 * mag[rows]
-        for name, got in (("first", first), ("second", second)):
+        for name, got in (("dg_fp8_gemm_nt", ref_entry), ("first noalloc", first), ("second noalloc", second)):
             g = _f64(got[rows])
             bad = ~(np.abs(g - r) <= tol)
             assert not bad.any(), (f"{M}x{N}x{K} sms={sms} {name} call: {bad.sum()} of {bad.size} outside "
-                                   f"tolerance; got={g[bad][:4]} ref={r[bad][:4]}")
+                                   f"tolerance; got={g[bad][:4]} oracle={r[bad][:4]}")
         assert dgm.dg_get_device_error() == 0
