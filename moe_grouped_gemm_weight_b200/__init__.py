@@ -40,7 +40,7 @@ class DGError(RuntimeError):
 class Plan(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int) for n in
                 ("block_m", "block_n", "stages", "m_blocks", "n_blocks", "tiles", "grid", "smem_bytes",
-                 "swap_ab", "split_k", "cta_pair", "tail_split")]
+                 "swap_ab", "split_k", "tail_split")]
 
     def as_dict(self) -> dict:
         return {n: getattr(self, n) for n, _ in self._fields_}

@@ -20,7 +20,6 @@
 #include "dg.h"
 #include "dg_kernel.cuh"
 #include "dg_kernel_small.cuh"
-#include "dg_kernel_pair.cuh"
 #include "dg_cast.cuh"
 #include "dg_kernel_ue8m0.cuh"
 
@@ -162,13 +161,7 @@ dg_status make_output_map(CUtensorMap* tm, void* base, int N, int rows, int grou
 struct Choice {
     int bn;
     int stages;
-    bool pair;
 };
-
-constexpr int kPairBN = 256;  // pair tile 256 x 256 (256 x 128 measured slower)
-constexpr int kPairStages = (227 * 1024 - 32 * 1024) / dg::PairCfg<kPairBN>::kStageBytes > 8
-                                ? 8
-                                : (227 * 1024 - 32 * 1024) / dg::PairCfg<kPairBN>::kStageBytes;
 
 // Ring depth: as many stages as fit in 227 KiB of shared memory, at most 8.
 template <int BN>
@@ -194,12 +187,10 @@ constexpr int smem_for() {
 // the DeepGEMM README page (section "非对齐的块大小"); here BN stays a
 // multiple of 64 so that the two promotion warpgroups split it into 32-column
 // TMEM loads.
-Choice choose(int m_blocks, int pair_m_blocks, int N, int num_sms, bool pair_ok, bool mn_major = false) {
-    // 192 (three promotion warpgroups) is measured ~12% slower per tile than
-    // 256 on the dense sweep: reachable with DG_FORCE_BN, not chosen.  An
-    // MN-major B is loaded in 128-wide atoms: tiles of 128 or 256 only.
+Choice choose(int m_blocks, int N, int num_sms, bool mn_major = false) {
+    // An MN-major B is loaded in 128-wide atoms: tiles of 128 or 256 only.
     const int cands[3] = {256, 128, 64};
-    Choice best{128, max_stages<128>(), false};
+    Choice best{128, max_stages<128>()};
     double best_cost = -1.0;
     for (int bn : cands) {
         if (mn_major && bn % 128 != 0) continue;
@@ -211,35 +202,12 @@ Choice choose(int m_blocks, int pair_m_blocks, int N, int num_sms, bool pair_ok,
             best.bn = bn;
         }
     }
-    // CTA pairs: a 256 x 256 tile on two SMs; per SM and K block the MMA work
-    // of a 128 x 256 tile with 32 KiB (128 + 128 rows) of operands.
-    if (pair_ok && num_sms >= 2) {
-        const int pair_tiles = pair_m_blocks * cdiv(N, kPairBN);
-        // per SM and K block: 128 x kPairBN MMA work, 128 + kPairBN/2 operand rows
-        const double mma = kPairBN, load = 0.75 * (128 + kPairBN / 2);
-        const double t_kb = mma > load ? mma : load;
-        const double cost = static_cast<double>(waves_cost(pair_tiles, num_sms / 2)) * t_kb;
-        best_cost = cost;
-        best.bn = kPairBN;
-        best.pair = true;
-    }
-    // DG_FORCE_BN=64|128|192|256 pins the single-CTA tile width (experiments).
-    const char* force_bn = std::getenv("DG_FORCE_BN");
-    if (force_bn && !best.pair) {
-        const int f = std::atoi(force_bn);
-        if (f == 128 || f == 256 || (!mn_major && (f == 64 || f == 192))) best.bn = f;
-    }
-    best.stages = best.pair ? kPairStages
-                            : best.bn == 256 ? max_stages<256>()
-                            : best.bn == 192 ? max_stages<192>()
-                            : best.bn == 128 ? max_stages<128>()
-                                             : max_stages<64>();
+    best.stages = best.bn == 256 ? max_stages<256>() : best.bn == 128 ? max_stages<128>() : max_stages<64>();
     return best;
 }
 
 int plan_smem(const Choice& c) {
-    if (c.pair) return dg::pair_smem_bytes<kPairBN, kPairStages>();
-    return c.bn == 256 ? smem_for<256>() : c.bn == 192 ? smem_for<192>() : c.bn == 128 ? smem_for<128>() : smem_for<64>();
+    return c.bn == 256 ? smem_for<256>() : c.bn == 128 ? smem_for<128>() : smem_for<64>();
 }
 
 dg_status check_sizes(int mode, int rows, int N, int K, int G) {
@@ -259,48 +227,95 @@ dg_status check_sizes(int mode, int rows, int N, int K, int G) {
 }
 
 // Few-row problems (dense M <= 128, masked M_max <= 256) go to the swap-AB
-// split-K kernel: TN activation rows per tile (masked: the smallest of
-// 32/64/128 that holds them; dense: see small_dense_tn), 128 weight rows per
-// tile, and K split over a cluster (small_split).  Per K block one CTA's loop
-// costs a fixed few hundred cycles (barrier hand-offs, MMA issue, the
-// promotion's TMEM round trips) that no deeper operand ring hides, so short
-// slices lose to their set-up and reduction.
+// kernel: 128 weight rows per tile, TN activation rows, one CTA per SM.
+// Tiles are spread over clusters of S CTAs that split K; without a split the
+// clusters are single CTAs that walk several tiles each.  small_choice picks
+// TN and S.
 bool use_small(int mode, int rows) { return (mode == 0 && rows <= 128) || (mode == 2 && rows <= 256); }
 
 int small_tn(int mode, int rows) {
-    const int t = mode == 2 ? (rows < 128 ? rows : 128) : rows;
+    const int t = rows < 128 ? rows : 128;
     return t <= 32 ? 32 : t <= 64 ? 64 : 128;
 }
 
-// K splits for `units` few-row tiles: as many as keep two CTAs on every SM
-// busy, at most kSmallMaxSplit slices of at least kSmallMinSliceKb K blocks.
-int small_split(long units, int nkb, int num_sms) {
-    constexpr int kSmallMinSliceKb = 8;
-    int split = static_cast<int>((2L * num_sms) / (units > 0 ? units : 1));
-    const int slices = nkb / kSmallMinSliceKb;
-    if (split > dg::kSmallMaxSplit) split = dg::kSmallMaxSplit;
-    if (split > slices) split = slices;
-    return split < 1 ? 1 : split;
+int small_max_split(int tn) {
+    return tn == 32 ? dg::SmallCfg<32>::kMaxSplit : tn == 64 ? dg::SmallCfg<64>::kMaxSplit : dg::SmallCfg<128>::kMaxSplit;
 }
 
-// Dense few-row calls may cut the activation rows into smaller tiles (TN / 2,
-// TN / 4, at least 32): more tiles, more CTAs in flight.  Per K block one
-// CTA's loop costs a roughly fixed time that grows with TN (measured with
-// clock stamps: about 0.44 / 0.56 / 0.75 us for TN = 32 / 64 / 128), so the
-// estimate is waves x K blocks per CTA x that cost; ties keep the larger TN.
-int small_dense_tn(int rows, int N, int nkb, int num_sms) {
-    const int tn0 = small_tn(0, rows);
-    int best_tn = tn0;
-    long best = -1;
-    for (int tn = tn0; tn >= 32; tn /= 2) {
-        const long units = static_cast<long>(cdiv(rows, tn)) * cdiv(N, 128);
-        const int split = small_split(units, nkb, num_sms);
-        const long waves = (units * split + 2L * num_sms - 1) / (2L * num_sms);
-        const long per_kb = tn == 32 ? 44 : tn == 64 ? 56 : 75;
-        const long cost = waves * ((nkb + split - 1) / split) * per_kb;
-        if (best < 0 || cost < best) { best = cost; best_tn = tn; }
+// CTAs of clusters of `s` one-CTA-per-SM blocks that can be resident at once
+// on `num_sms` SMs.  Clusters are placed inside GPCs, so large clusters leave
+// SMs unused; measured on a 148-SM B200 with cudaOccupancyMaxActiveClusters
+// (227 KiB of shared memory per CTA), scaled down for a smaller SM budget.
+int small_cluster_capacity(int s, int num_sms) {
+    static const int kB200[9] = {0, 148, 148, 135, 132, 130, 132, 105, 120};
+    if (s < 1 || s > 8) return 0;
+    const int cap = static_cast<int>(static_cast<long long>(kB200[s]) * num_sms / 148);
+    return cap - cap % s;
+}
+
+// Estimated time (us) of a few-row launch with TN activation rows per tile
+// and K split into `split` slices.  Fitted to CUDA-graph timings of the 12
+// dense decode shapes of the sweep under 41 (TN, split) choices on a 148-SM
+// B200 (rms error about 1 us); it picks the fastest measured choice, or one
+// within 4 %, on every shape.  Terms: a fixed cost (launch, set-up, first
+// loads); the longest CTA's K loop -- bound by its per-K-block pipeline cost,
+// by its own operand stream (about 80 GB/s per CTA), or by the whole weight
+// stream at HBM speed; the split reduction; an epilogue per tile.
+double small_cost(long tiles, int nkb, int tn, int split, int num_sms, double weight_bytes) {
+    constexpr double kFixedUs = 3.9, kReduceUs = 2.3, kTileUs = 0.58, kCtaGBs = 81.5, kHbmGBs = 6500.0;
+    const double per_kb = tn == 32 ? 0.218 : tn == 64 ? 0.257 : 0.47;
+    long kb_per_cta, tiles_per_cta;
+    if (split > 1) {
+        kb_per_cta = (nkb + split - 1) / split;
+        tiles_per_cta = 1;
+    } else {
+        tiles_per_cta = (tiles + num_sms - 1) / num_sms;
+        kb_per_cta = static_cast<long>(nkb) * tiles_per_cta;
     }
-    return best_tn;
+    const double loop = static_cast<double>(kb_per_cta) * per_kb;
+    const double stream = static_cast<double>(kb_per_cta) * (128.0 + tn) * dg::kBK / (kCtaGBs * 1e3);
+    const double hbm = weight_bytes / (kHbmGBs * 1e3);
+    double t = loop > stream ? loop : stream;
+    t = t > hbm ? t : hbm;
+    return kFixedUs + t + (split > 1 ? kReduceUs : 0.0) + kTileUs * static_cast<double>(tiles_per_cta);
+}
+
+struct SmallChoice {
+    int tn;
+    int split;
+};
+
+// Tile height and K split of a few-row launch: the (TN, split) of least
+// small_cost among TN in {32, 64, 128} no taller than the rows need (a
+// shorter TN reads each weight tile once per TN-row block, from L2 after the
+// first) and splits that keep at least kSmallMinSliceKb K blocks per slice,
+// whose clusters all fit on the GPU at once, used only while the tiles alone
+// leave SMs idle.  `rows` is the row count that decides the TN-row blocks
+// (masked: the expected rows per group); `all_rows` the most a group can
+// have, which the launch must cover.
+SmallChoice small_choice(int rows, int all_rows, int G, int N, int K, int num_sms) {
+    constexpr int kSmallMinSliceKb = 4;
+    const int nkb = K / dg::kBK;
+    const int n_blocks = cdiv(N, 128);
+    const double weight_bytes = static_cast<double>(G) * N * K;
+    const int tn_max = small_tn(0, all_rows);
+    SmallChoice best{tn_max, 1};
+    double best_t = -1.0;
+    for (int tn = tn_max; tn >= 32; tn /= 2) {
+        const long tiles = static_cast<long>(G) * cdiv(rows, tn) * n_blocks;
+        const long all_tiles = static_cast<long>(G) * cdiv(all_rows, tn) * n_blocks;
+        for (int split = 1; split <= small_max_split(tn); ++split) {
+            if (split > 1 && (all_tiles >= num_sms || nkb / split < kSmallMinSliceKb ||
+                              all_tiles * split > small_cluster_capacity(split, num_sms)))
+                continue;
+            const double t = small_cost(tiles, nkb, tn, split, num_sms, weight_bytes);
+            if (best_t < 0 || t < best_t - 1e-9) {
+                best_t = t;
+                best = {tn, split};
+            }
+        }
+    }
+    return best;
 }
 
 int small_smem(int tn) {
@@ -318,57 +333,33 @@ dg_status plan(int mode, int rows, int N, int K, int G, int num_sms, dg_plan* ou
     if (num_sms <= 0) return fail(DG_ERR_INVALID_ARG, "num_sms must be positive");
     *out = dg_plan{};
     if (layout == 0 && use_small(mode, rows)) {
-        const int tn = mode == 0 ? small_dense_tn(rows, N, K / dg::kBK, num_sms) : small_tn(mode, rows);
+        // Masked: tiles past masked_m are skipped on the device; with a hint,
+        // count only the tiles expected to hold rows.
+        const int expect = (mode == 2 && expected_m > 0 && expected_m < rows) ? expected_m : rows;
+        const SmallChoice ch = small_choice(expect, rows, mode == 2 ? G : 1, N, K, num_sms);
+        const int tn = ch.tn, split = ch.split;
         const int per_group = cdiv(rows, tn);
         const int m_blocks = mode == 2 ? G * per_group : per_group;
         const int n_blocks = cdiv(N, 128);
-        // Masked: tiles past masked_m exit at once; with a hint, count only the
-        // tiles expected to hold rows.
-        int active_m = m_blocks;
-        if (mode == 2 && expected_m > 0) active_m = G * cdiv(expected_m < rows ? expected_m : rows, tn);
-        const long units = static_cast<long>(active_m) * n_blocks;
-        const int split = small_split(units, K / dg::kBK, num_sms);
         out->block_m = tn;
         out->block_n = 128;
         out->stages = small_stages(tn);
         out->m_blocks = m_blocks;
         out->n_blocks = n_blocks;
         out->tiles = m_blocks * n_blocks;
-        out->grid = out->tiles * split;
+        // Split: one cluster per tile (the host tile count is an upper bound
+        // of the device's for masked calls).  Unsplit: persistent, at most
+        // one CTA per SM.
+        const long all = static_cast<long>(m_blocks) * n_blocks;
+        out->grid = split > 1 ? static_cast<int>(all * split) : static_cast<int>(all < num_sms ? all : num_sms);
         out->smem_bytes = small_smem(tn);
         out->swap_ab = 1;
         out->split_k = split;
-        out->cta_pair = 0;
         out->tail_split = 1;  // the cluster split replaces the tail split
         return DG_OK;
     }
     const int m_blocks = (mode == 2) ? G * cdiv(rows, dg::kBM) : cdiv(rows, dg::kBM);
-    // Pairs need every 256-row tile inside one group: dense, or masked (groups
-    // are separate blocks of M_max rows); not the contiguous layout, whose
-    // segments are only 128-row aligned.
-    // CTA pairs are measured no faster than single-CTA 128 x 256 tiles on the
-    // dense sweep, so they are used only when DG_FORCE_PAIR=1 (experiments).
-    const char* force_pair = std::getenv("DG_FORCE_PAIR");
-    const bool pairs = force_pair && force_pair[0] == '1' && mode != 1 && layout == 0;
-    const int pair_m_blocks = (mode == 2 ? G : 1) * cdiv(rows, dg::kPairBM);
-    const Choice c = choose(m_blocks, pair_m_blocks, N, num_sms, pairs, layout != 0);
-    if (c.pair) {
-        const int per_group = cdiv(rows, dg::kPairBM);
-        out->block_m = dg::kPairBM;
-        out->block_n = kPairBN;
-        out->stages = c.stages;
-        out->m_blocks = mode == 2 ? G * per_group : per_group;
-        out->n_blocks = cdiv(N, kPairBN);
-        out->tiles = out->m_blocks * out->n_blocks;
-        const int pairs = num_sms / 2;
-        out->grid = 2 * ((mode == 2 || out->tiles > pairs) ? pairs : out->tiles);
-        out->smem_bytes = plan_smem(c);
-        out->swap_ab = 0;
-        out->split_k = 1;
-        out->cta_pair = 1;
-        out->tail_split = 1;  // pair tiles have no K-split tail
-        return DG_OK;
-    }
+    const Choice c = choose(m_blocks, N, num_sms, layout != 0);
     out->block_m = dg::kBM;
     out->block_n = c.bn;
     out->stages = c.stages;
@@ -379,7 +370,6 @@ dg_status plan(int mode, int rows, int N, int K, int G, int num_sms, dg_plan* ou
     out->smem_bytes = plan_smem(c);
     out->swap_ab = 0;
     out->split_k = 1;
-    out->cta_pair = 0;
     out->tail_split = 1;
     // Dense: when the last wave is partial (R leftover tiles after W full
     // waves), split each leftover tile into S K slices run by the idle CTAs.
@@ -405,21 +395,21 @@ dg_status plan(int mode, int rows, int N, int K, int G, int num_sms, dg_plan* ou
 
 // ------------------------------------------------------------ launch ----
 
-// With DG_PDL=1 every GEMM launch allows programmatic dependent launch: the
-// kernel's set-up (barriers, TMEM, tensor-map and weight prefetch) may overlap
-// the end of the previous kernel in the stream; the kernels always wait
-// (griddepcontrol.wait) before touching global data.  It is off by default:
-// measured in CUDA-graph replays it shortens some decode-sized launches (e.g.
-// 64x32768x512 by about a quarter) but lengthens cluster launches with large
-// grids (64x7168x16384 by up to a third), whose CTAs are then placed into
-// slots as the previous grid frees them instead of spread over an idle GPU.
+// Every launch allows programmatic dependent launch unless DG_PDL=0 (or
+// dg_set_pdl(0)): the kernel's set-up (barriers, TMEM, tensor-map prefetch)
+// may overlap the end of the previous kernel in the stream; the kernels always
+// wait (griddepcontrol.wait) before touching global data.  Measured in
+// CUDA-graph replays of back-to-back GEMMs it saves about 1 us per decode-sized
+// launch (e.g. 64x32768x512: 9.7 -> 8.2 us) and 1-2 % on the large shapes;
+// every GEMM kernel takes one CTA per SM, so a dependent grid's CTAs start on
+// SMs as the previous grid leaves them.
 std::atomic<int> g_pdl{-1};  // -1: from DG_PDL, else 0 / 1 from dg_set_pdl
 
 bool pdl_enabled() {
     const int set = g_pdl.load();
     if (set >= 0) return set != 0;
     const char* v = std::getenv("DG_PDL");
-    return v && v[0] == '1';
+    return !(v && v[0] == '0');
 }
 
 void set_pdl(cudaLaunchAttribute& a) {
@@ -456,83 +446,10 @@ dg_status launch_one(const dg::Params& p, const CUtensorMap& ta, const CUtensorM
     return ok();
 }
 
-// How many 2-CTA clusters of the pair kernel can be resident at once (a
-// cluster must fit inside one GPC, so this can be below SMs / 2).  Cached per
-// device; 0 if the query fails.
-template <int MODE>
-int pair_max_active_clusters() {
-    static std::atomic<int> cached[kMaxDevices];
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 0;
-    int n = cached[dev].load();
-    if (n > 0) return n;
-    constexpr int smem = dg::pair_smem_bytes<kPairBN, kPairStages>();
-    auto kern = dg::fp8_gemm_pair_kernel<kPairBN, kPairStages, MODE>;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) {
-        cudaGetLastError();
-        return 0;
-    }
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(2 * 74, 1, 1);
-    cfg.blockDim = dim3(dg::kThreads, 1, 1);
-    cfg.dynamicSmemBytes = smem;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) {
-        cudaGetLastError();
-        return 0;
-    }
-    cached[dev].store(n);
-    return n;
-}
-
-template <int MODE>
-dg_status launch_pair(const dg::Params& p, const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& td,
-                      const dg_plan& pl, cudaStream_t stream) {
-    constexpr int smem = dg::pair_smem_bytes<kPairBN, kPairStages>();
-    static_assert(smem <= 227 * 1024, "shared memory budget exceeded");
-    auto kern = dg::fp8_gemm_pair_kernel<kPairBN, kPairStages, MODE>;
-    static std::atomic<int> attr_set[kMaxDevices];
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev >= 0 && dev < kMaxDevices && !attr_set[dev].load()) {
-        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-            return fail(DG_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(cudaGetLastError()));
-        attr_set[dev].store(1);
-    }
-    // Persistent grid: never more clusters than can be resident together.
-    int grid = pl.grid;
-    const int max_clusters = pair_max_active_clusters<MODE>();
-    if (max_clusters > 0 && grid > 2 * max_clusters) grid = 2 * max_clusters;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
-    cfg.blockDim = dim3(dg::kThreads, 1, 1);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[2];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    set_pdl(attr[1]);
-    cfg.numAttrs = 2;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, kern, p, ta, tb, td);
-    if (e == cudaSuccess) e = cudaGetLastError();
-    if (e != cudaSuccess) return fail(DG_ERR_CUDA, "kernel launch failed: %s", cudaGetErrorString(e));
-    return ok();
-}
-
 template <int TN, int MODE>
 dg_status launch_small(const dg::Params& p, const CUtensorMap& ta, const CUtensorMap& tb, const dg_plan& pl,
                        cudaStream_t stream) {
     constexpr int smem = dg::small_smem_bytes<TN>();
-    static_assert(smem <= 113 * 1024, "two CTAs per SM need <= 113 KiB each");
     auto kern = dg::fp8_gemm_swapab_kernel<TN, MODE>;
     static std::atomic<int> attr_set[kMaxDevices];
     int dev = 0;
@@ -543,8 +460,7 @@ dg_status launch_small(const dg::Params& p, const CUtensorMap& ta, const CUtenso
         attr_set[dev].store(1);
     }
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(pl.split_k), static_cast<unsigned>(pl.n_blocks),
-                       static_cast<unsigned>(pl.m_blocks));
+    cfg.gridDim = dim3(static_cast<unsigned>(pl.grid), 1, 1);
     cfg.blockDim = dim3(dg::kSmallThreads, 1, 1);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
@@ -578,7 +494,6 @@ dg_status dispatch(const dg_plan& pl, const dg::Params& p, const CUtensorMap& ta
                    const CUtensorMap& td, cudaStream_t stream) {
     switch (pl.block_n) {
         case 256: return launch_one<256, max_stages<256>(), MODE>(p, ta, tb, td, pl.grid, stream);
-        case 192: return launch_one<192, max_stages<192>(), MODE>(p, ta, tb, td, pl.grid, stream);
         case 128: return launch_one<128, max_stages<128>(), MODE>(p, ta, tb, td, pl.grid, stream);
         case 64: return launch_one<64, max_stages<64>(), MODE>(p, ta, tb, td, pl.grid, stream);
         default: return fail(DG_ERR_UNSUPPORTED, "no kernel for block_n=%d", pl.block_n);
@@ -750,7 +665,7 @@ dg::Params make_params(uint16_t* D, const float* sa, int sa_stride, const float*
     p.m_blocks = pl.m_blocks;
     p.raster = pl.swap_ab ? 1
                           : choose_raster(pl.m_blocks, pl.n_blocks, pl.block_m, pl.block_n, K,
-                                          pl.cta_pair ? pl.grid / 2 : pl.grid);
+                                          pl.grid);
     p.b_stream = 0;
     p.tail_split = 1;
     p.full_tiles = pl.tiles;
@@ -814,7 +729,7 @@ dg_status k_grouped(uint16_t* D, const uint8_t* A, const float* sa, int sa_strid
     const int sms = effective_sms();
     if (sms <= 0) return fail(DG_ERR_CUDA, "no CUDA device");
     const int m_blocks = cdiv(M, dg::kBM);
-    const Choice c = choose(G * m_blocks, 0, N, sms, false, true);
+    const Choice c = choose(G * m_blocks, N, sms, true);
     dg_plan pl{};
     pl.block_m = dg::kBM;
     pl.block_n = c.bn;
@@ -902,15 +817,15 @@ dg_status dg_fp8_gemm_nt(uint16_t* D, const uint8_t* A, const float* sa, int sa_
         if ((s = make_operand_map(&ta, A, K, M, 1, pl.block_m, false)) != DG_OK) return s;
         if ((s = make_operand_map(&tb, B, K, N, 1, 128, true)) != DG_OK) return s;
         dg::Params p = make_params(D, sa, sa_stride, sb, M, N, K, 1, pl);
+        p.b_stream = pl.m_blocks == 1;
         return dispatch_small<dg::kDense>(pl, p, ta, tb, static_cast<cudaStream_t>(stream));
     }
     if ((s = make_operand_map(&ta, A, K, M, 1, dg::kBM, false)) != DG_OK) return s;
-    if ((s = make_operand_map(&tb, B, K, N, 1, pl.cta_pair ? pl.block_n / 2 : pl.block_n, true)) != DG_OK) return s;
+    if ((s = make_operand_map(&tb, B, K, N, 1, pl.block_n, true)) != DG_OK) return s;
     CUtensorMap td;
     if ((s = make_output_map(&td, D, N, M, 1, false)) != DG_OK) return s;
     dg::Params p = make_params(D, sa, sa_stride, sb, M, N, K, 1, pl);
     p.b_stream = pl.m_blocks == 1;
-    if (pl.cta_pair) return launch_pair<dg::kDense>(p, ta, tb, td, pl, static_cast<cudaStream_t>(stream));
     TailWorkspace ws;
     if (pl.tail_split > 1 && tail_workspace(static_cast<cudaStream_t>(stream), &ws)) {
         p.tail_split = pl.tail_split;
@@ -939,15 +854,15 @@ dg_status dg_fp8_gemm_nt_noalloc(uint16_t* D, const uint8_t* A, const float* sa,
         if ((s = make_operand_map(&ta, A, K, M, 1, pl.block_m, false)) != DG_OK) return s;
         if ((s = make_operand_map(&tb, B, K, N, 1, 128, true)) != DG_OK) return s;
         dg::Params p = make_params(D, sa, sa_stride, sb, M, N, K, 1, pl);
+        p.b_stream = pl.m_blocks == 1;
         return dispatch_small<dg::kDense>(pl, p, ta, tb, st);
     }
     if ((s = make_operand_map(&ta, A, K, M, 1, dg::kBM, false)) != DG_OK) return s;
-    if ((s = make_operand_map(&tb, B, K, N, 1, pl.cta_pair ? pl.block_n / 2 : pl.block_n, true)) != DG_OK) return s;
+    if ((s = make_operand_map(&tb, B, K, N, 1, pl.block_n, true)) != DG_OK) return s;
     CUtensorMap td;
     if ((s = make_output_map(&td, D, N, M, 1, false)) != DG_OK) return s;
     dg::Params p = make_params(D, sa, sa_stride, sb, M, N, K, 1, pl);
     p.b_stream = pl.m_blocks == 1;
-    if (pl.cta_pair) return launch_pair<dg::kDense>(p, ta, tb, td, pl, st);
     if (pl.tail_split > 1) {
         // One partial per (tail tile, slice >= 1) and one flag per partial.
         const int full = (pl.tiles / pl.grid) * pl.grid;
@@ -1100,16 +1015,16 @@ dg_status dg_grouped_masked_nt(uint16_t* D, const uint8_t* A, const float* sa, i
         dg::Params p = make_params(D, sa, sa_stride, sb, M_max, N, K, G, pl);
         p.masked_m = masked_m;
         p.m_blocks = pl.m_blocks / G;  // TN-row blocks per group
+        p.b_stream = p.m_blocks == 1;
         return dispatch_small<dg::kMasked>(pl, p, ta, tb, static_cast<cudaStream_t>(stream));
     }
     if ((s = make_operand_map(&ta, A, K, M_max, G, dg::kBM, true)) != DG_OK) return s;
-    if ((s = make_operand_map(&tb, B, K, N, G, pl.cta_pair ? pl.block_n / 2 : pl.block_n, true)) != DG_OK) return s;
+    if ((s = make_operand_map(&tb, B, K, N, G, pl.block_n, true)) != DG_OK) return s;
     CUtensorMap td;
     if ((s = make_output_map(&td, D, N, M_max, G, true)) != DG_OK) return s;
     dg::Params p = make_params(D, sa, sa_stride, sb, M_max, N, K, G, pl);
     p.masked_m = masked_m;
     p.b_stream = M_max <= dg::kBM;
-    if (pl.cta_pair) return launch_pair<dg::kMasked>(p, ta, tb, td, pl, static_cast<cudaStream_t>(stream));
     return dispatch<dg::kMasked>(pl, p, ta, tb, td, static_cast<cudaStream_t>(stream));
 }
 

@@ -5,9 +5,10 @@
 //   * warp 0 (operand producer): TMA-loads, for every 128-wide K block kb,
 //     the A tile [128 rows x 128 K] and the B tile [BN rows x 128 K]
 //     (128-byte swizzle) into a STAGES-deep shared-memory ring.
-//   * warp 1 (MMA): issues four tcgen05.mma kind::f8f6f4 (K = 32 each) that
-//     write P_kb = A_kb . B_kb^T into a FRESH TMEM buffer (one of NBUF), then
-//     commits to the ring's "empty" barrier and the buffer's "full" barrier.
+//   * warps 1 and 3 (MMA, alternate K blocks): issue four tcgen05.mma
+//     kind::f8f6f4 (K = 32 each) that write P_kb = A_kb . B_kb^T into a FRESH
+//     TMEM buffer (one of NBUF), then commit to the ring's "empty" barrier and
+//     the buffer's "full" barrier.
 //   * warp 2 (scale producer): copies sa[m0..m0+127, kb] and the one or two
 //     sb[n/128, kb] the tile needs into a 16-deep shared-memory scale ring,
 //     running ahead of the promotion so that no global-memory latency sits on
@@ -244,8 +245,8 @@ fp8_gemm_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtens
     uint64_t* tempty = tfull + kNBuf;
     uint64_t* sfull = tempty + kNBuf;
     uint64_t* sempty = sfull + kScaleSlots;
-    uint64_t* done = sempty + kScaleSlots;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+    uint64_t* done = sempty + kScaleSlots;  // one per MMA warp
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 2);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
     float* sring = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(full) + 512);
     int* mb_prefix = reinterpret_cast<int*>(sring + kScaleSlots * kScaleSlotFloats);
@@ -267,6 +268,7 @@ fp8_gemm_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtens
             mbar_init(sempty + s, C::kEpiWarpsC);
         }
         mbar_init(done, 1);
+        mbar_init(done + 1, 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -371,18 +373,28 @@ fp8_gemm_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtens
                 mbar_wait_drain(full + (i % STAGES), static_cast<uint32_t>((i / STAGES) & 1));
         }
         __syncwarp();
-    } else if (warp == 1) {
+    } else if (warp == 1 || warp == 3) {
         // ----------------------------------------------------------- MMA ----
+        // Two warps issue the MMAs of alternate K blocks (the CTA's i-th K
+        // block goes to warp 1 for even i, to warp 3 for odd i).  Issuing a
+        // block's four tcgen05.mma and two commits keeps a warp busy for
+        // several hundred cycles; with two issuers one of them is always
+        // already waiting for the next free TMEM buffer, so the tensor core
+        // gets the next block as soon as the promotion releases it.
         constexpr uint32_t idesc = idesc_e4m3_f32_major(kBM, BN, kAmn, kBmn);
-        int stage = 0, buf = 0;
-        uint32_t phase = 0, bphase = 0;
+        const int mw = warp == 1 ? 0 : 1;
+        int i = 0;  // K blocks of this CTA so far, over all its work
         bool ok = true;
         Work w;
         for (int it = 0; ok && next_work(p, tiles, it, w); ++it) {
             const Tile tl = decode_tile<BN, MODE>(p, w.t, m_blocks, mb_prefix);
             if (!tl.valid) continue;
             group_k_range<MODE>(p, tl, w);
-            for (int kb = w.kb0; kb < w.kb1; ++kb) {
+            for (int kb = w.kb0; kb < w.kb1; ++kb, ++i) {
+                if ((i & 1) != mw) continue;
+                const int stage = i % STAGES, buf = i % kNBuf;
+                const uint32_t phase = static_cast<uint32_t>(i / STAGES) & 1u;
+                const uint32_t bphase = static_cast<uint32_t>(i / kNBuf) & 1u;
                 if (!mbar_wait(tempty + buf, bphase ^ 1u, abort_flag)) { ok = false; break; }
                 if (!mbar_wait(full + stage, phase, abort_flag)) { ok = false; break; }
                 tc_fence_after();
@@ -402,14 +414,12 @@ fp8_gemm_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtens
                     umma_commit(tfull + buf);
                 }
                 __syncwarp();
-                if (++stage == STAGES) { stage = 0; phase ^= 1u; }
-                if (++buf == kNBuf) { buf = 0; bphase ^= 1u; }
             }
         }
-        // All MMAs of this CTA must have finished before TMEM is released.
+        // All MMAs of this warp must have finished before TMEM is released.
         if (lane == 0) {
-            umma_commit(done);
-            mbar_wait_drain(done, 0);
+            umma_commit(done + mw);
+            mbar_wait_drain(done + mw, 0);
         }
         __syncwarp();
     } else if (warp == 2) {

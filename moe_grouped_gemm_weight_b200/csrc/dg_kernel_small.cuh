@@ -1,95 +1,151 @@
 // dg_kernel_small.cuh -- sm_100a kernel for few rows per group (decode-sized M).
 //
-// With M <= 128 rows the output has too few 128-row tiles to keep 148 SMs
-// streaming the weights, so this kernel swaps the operands and splits K:
-//   * the MMA's 128-row side runs over N (the weights B), its N side over the
-//     TN (32, 64 or 128) rows of A:  P_kb^T[n, m] = sum_k B[n,k] * A[m,k];
-//   * a thread-block cluster of S CTAs shares one 128 x TN output tile; CTA r
-//     of the cluster handles K blocks [r*nkb/S, (r+1)*nkb/S);
-//   * each CTA promotes its blocks into FP32 registers exactly as the large
-//     kernel does, acc[n,m] += (sa[m,kb] * sb[n/128,kb]) * P_kb[n,m] (the
-//     128-row weight tile lies inside one 128x128 scale block, so sb is one
-//     value per kb), with sa*sb formed once per kb by the scale warp;
-//   * the S partial tiles are added in a fixed order (CTA 0 first) through
-//     distributed shared memory -- no global scratch -- and the sum is rounded
-//     to bf16 once and stored.
-// Per CTA: 256 threads, <= 113 KiB shared memory and 256 TMEM columns, so two
-// CTAs share an SM and every SM keeps up to 2 x STAGES K blocks in flight.
+// With M <= 128 rows the GEMM streams the weights B once from HBM and the
+// activations are a small, L2-resident operand.  The kernel is built around
+// keeping every SM's TMA queue full of weight tiles from the first
+// microsecond to the last:
+//   * operands swapped: the MMA's 128-row side runs over 128 weight rows,
+//     its N side over the TN (32, 64 or 128) activation rows, so one tile
+//     covers all rows of a group and B is read exactly once;
+//   * one CTA per SM with a deep operand ring (5 to 10 stages, up to ~200
+//     KiB in flight), so few round trips to HBM cover a CTA's share;
+//   * tiles (group, TN-row block, 128-wide block of N) are spread over
+//     clusters of S CTAs; CTA r of a cluster handles K blocks
+//     [r*nkb/S, (r+1)*nkb/S) of its cluster's tile.  S = 1 clusters are
+//     persistent (a CTA walks tiles cid, cid + C, ... with one ring across
+//     them); S > 1 is used only when every cluster has one tile, and the host
+//     sizes S so that all clusters are resident at once;
+//   * each CTA promotes its K blocks in FP32 registers,
+//         acc[n, m] += (sa[m, kb] * sb[n/128, kb]) * P_kb[n, m],
+//     with two promotion warpgroups splitting the activation rows (the
+//     128-row weight tile lies inside one 128 x 128 scale block, so sb is one
+//     value per K block);
+//   * split tiles are reduced through distributed shared memory without a
+//     barrier on the critical path: each CTA writes its FP32 partial tile into
+//     its (now idle) ring and bulk-copies slice r of it into CTA r's receive
+//     area, counted on CTA r's mbarrier; CTA r then adds the S slices in rank
+//     order (a fixed order, so results are deterministic), rounds to bf16 once
+//     and stores its rows.  Unsplit tiles are rounded to bf16, staged in
+//     shared memory and stored with 16-byte writes.
 // Warp roles: 0 TMA producer, 1 TMEM owner + MMA issuer, 2 scale producer,
-// 3 idle, 4..7 promotion (TMEM lane quarter = warp % 4, lane = output column).
+// 3 second MMA issuer, 4..11 promotion (warpgroup h = activation rows [h*TN/2, (h+1)*TN/2),
+// TMEM lane quarter = warp % 4, lane = weight row).
 #pragma once
 
 #include "dg_kernel.cuh"
 
 namespace dg {
 
-constexpr int kSmallThreads = 256;
+constexpr int kSmallThreads = 384;
 constexpr int kSmallFirstEpiWarp = 4;
-constexpr int kSmallEpiWarps = 4;
+constexpr int kSmallEpiWarps = 8;
+constexpr int kSmallEpiThreads = 32 * kSmallEpiWarps;
 constexpr int kSmallScaleSlots = 16;  // depth of the scale ring, in K blocks
 // The scale ring is filled and released kSmallScaleGroup K blocks at a time,
 // so the promotion waits on a scale barrier once per group.
 constexpr int kSmallScaleGroup = 4;
 constexpr int kSmallScaleGroups = kSmallScaleSlots / kSmallScaleGroup;
-constexpr int kSmallTmemCols = 256;
-// Largest cluster (K splits per tile).  Measured on the M = 64 / 128 shapes of
-// the dense sweep, clusters of 6 and 8 CTAs were never faster than 4: at two
-// CTAs per SM an 8-CTA cluster lands on four SMs, and per slice the set-up and
-// the DSMEM reduction cost more than the shorter K loop saves.
-constexpr int kSmallMaxSplit = 4;
+constexpr int kSmallSmemLimit = 232448;  // 227 KiB: one CTA per SM
+constexpr int kSmallBarrierBytes = 1024;
+constexpr int kSmallGroupTableBytes = 8 * (kMaxMaskedGroups + 1);  // masked: tile prefix + clamped counts
+
+// Largest receive area over the cluster sizes a TN allows: S - 1 slices of
+// ceil(TN / S) rows of 128 FP32 values.
+constexpr int small_recv_bytes(int tn, int max_split) {
+    int best = 0;
+    for (int s = 2; s <= max_split; ++s) {
+        const int b = (s - 1) * ((tn + s - 1) / s) * 128 * 4;
+        best = b > best ? b : best;
+    }
+    return best;
+}
 
 template <int TN>
 struct SmallCfg {
     static_assert(TN == 32 || TN == 64 || TN == 128, "TN must be 32, 64 or 128");
-    static constexpr int kTileBBytes = 128 * kBK;   // 128 weight rows
-    static constexpr int kTileABytes = TN * kBK;    // TN activation rows
+    static constexpr int kMaxSplit = TN == 128 ? 4 : 8;  // cluster size (K slices per tile)
+    static constexpr int kTileBBytes = 128 * kBK;        // 128 weight rows
+    static constexpr int kTileABytes = TN * kBK;         // TN activation rows
     static constexpr int kStageBytes = kTileBBytes + kTileABytes;
-    static constexpr int kStages = (96 * 1024) / kStageBytes;  // 4, 4 or 3 stages: ~96 KiB of ring
-    static constexpr int kNBuf = kSmallTmemCols / TN > 4 ? 4 : kSmallTmemCols / TN;
-    static constexpr int kChunks = TN / 32;
-    static constexpr int kBatch = TN == 128 ? 1 : (kChunks < 2 ? kChunks : 2);
-    static constexpr int kRedBytes = TN * 128 * 4;  // FP32 partial tile, aliases the ring
-    static_assert(kRedBytes <= kStages * kStageBytes, "partial tile must fit in the ring");
-    static_assert(kNBuf * TN <= kSmallTmemCols, "TMEM buffers overflow the allocation");
+    static constexpr int kTileF32Bytes = TN * 128 * 4;   // FP32 partial tile
+    static constexpr int kRecvBytes = small_recv_bytes(TN, kMaxSplit);
+    static constexpr int kStageOutBytes = TN * 128 * 2;  // bf16 tile staged for the store
+    static constexpr int kAuxBytes = kRecvBytes > kStageOutBytes ? kRecvBytes : kStageOutBytes;
+    static constexpr int kScaleBytes = kSmallScaleSlots * (TN + 4) * 4;
+    static constexpr int kFixedBytes = 1024 + kAuxBytes + kScaleBytes + kSmallBarrierBytes + kSmallGroupTableBytes;
+    static constexpr int kStagesFit = (kSmallSmemLimit - kFixedBytes) / kStageBytes;
+    static constexpr int kStages = kStagesFit > 12 ? 12 : kStagesFit;
+    static constexpr int kNBuf = 4;                       // TMEM partial buffers
+    static constexpr int kTmemCols = kNBuf * TN <= 128 ? 128 : (kNBuf * TN <= 256 ? 256 : 512);
+    static constexpr int kCols = TN / 2;                  // activation rows per promotion warpgroup
+    static constexpr int kChunk = kCols < 32 ? kCols : 32;  // columns per tcgen05.ld
+    static constexpr int kChunks = kCols / kChunk;
+    static_assert(kTileF32Bytes <= kStages * kStageBytes, "partial tile must fit in the ring");
+    static_assert(kStages >= 4, "ring too shallow");
+    static_assert(kStages * kStageBytes + kFixedBytes <= kSmallSmemLimit, "shared memory overflow");
 };
 
 template <int TN>
 constexpr int small_smem_bytes() {
-    return 1024 + SmallCfg<TN>::kStages * SmallCfg<TN>::kStageBytes + 512 + kSmallScaleSlots * (TN + 4) * 4;
+    return SmallCfg<TN>::kStages * SmallCfg<TN>::kStageBytes + SmallCfg<TN>::kFixedBytes;
 }
 
-// Grid: x = split index (the cluster spans x), y = 128-wide block of N,
-// z = TN-row block of M (masked: g * m_blocks + block inside the group;
-// Params::m_blocks holds the blocks per group).
+// One tile of the few-row kernel.
+struct SmallTile {
+    int g;     // group
+    int m0;    // first activation row inside the group
+    int n0;    // first weight row (output column)
+    int rows;  // rows of the group that exist (dense M, masked masked_m[g])
+};
+
+// Tile t in the order (group, n-block, m-block), m-block fastest: tiles that
+// run on neighbouring clusters share their weight tiles in L2.
 template <int TN, int MODE>
-__global__ void __launch_bounds__(kSmallThreads, 2)
+__device__ __forceinline__ SmallTile small_tile(const Params& p, int t, const int* prefix, const int* counts) {
+    SmallTile tl;
+    if (MODE == kMasked) {
+        int lo = 0, hi = p.G - 1;  // largest g with prefix[g] <= t
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (prefix[mid] <= t) lo = mid; else hi = mid - 1;
+        }
+        const int local = t - prefix[lo];
+        const int mbg = (counts[lo] + TN - 1) / TN;
+        tl.g = lo;
+        tl.n0 = (local / mbg) * 128;
+        tl.m0 = (local % mbg) * TN;
+        tl.rows = counts[lo];
+    } else {
+        tl.g = 0;
+        tl.n0 = (t / p.m_blocks) * 128;
+        tl.m0 = (t % p.m_blocks) * TN;
+        tl.rows = p.M;
+    }
+    return tl;
+}
+
+// Grid: 1-D, clusters of S CTAs along x (S = cluster size).  Params::m_blocks
+// holds the TN-row blocks per group; Params::n_blocks the 128-wide blocks of N.
+template <int TN, int MODE>
+__global__ void __launch_bounds__(kSmallThreads, 1)
 fp8_gemm_swapab_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtensorMap tmA,
                        const __grid_constant__ CUtensorMap tmB) {
     using C = SmallCfg<TN>;
     constexpr int STAGES = C::kStages;
     constexpr int kNBuf = C::kNBuf;
-
-    const int S = gridDim.x;
-    const int rank = blockIdx.x;
-    const int n0 = blockIdx.y * 128;
-    int g = 0, m0;
-    if (MODE == kMasked) {
-        g = blockIdx.z / p.m_blocks;
-        m0 = (blockIdx.z % p.m_blocks) * TN;
-    } else {
-        m0 = blockIdx.z * TN;
+    // The tensor maps live in parameter space: start fetching them first.
+    if (threadIdx.x == 0) {
+        prefetch_tmap(&tmA);
+        prefetch_tmap(&tmB);
     }
-    int rows_valid = p.M;
-    if (MODE == kMasked) {
-        // masked_m may come from the previous kernel in the stream.
-        griddep_wait();
-        const int mm = __ldg(p.masked_m + g);
-        if ((mm < 0 || mm > p.M) && rank == 0 && blockIdx.y == 0 && m0 == 0) atomicOr(&g_dg_error, 4u);
-        rows_valid = min(max(mm, 0), p.M);
-    }
-    // Every CTA of a cluster shares (y, z), so the whole cluster leaves together.
-    if (m0 >= rows_valid) return;
 
+    const int S = static_cast<int>(cluster_nctarank());
+    const int rank = static_cast<int>(cluster_ctarank());
+    const int cid = static_cast<int>(blockIdx.x) / S;
+    const int nclusters = static_cast<int>(gridDim.x) / S;
+    // Split clusters own one tile each (the host launches one cluster per
+    // tile); single-CTA clusters walk tiles cid, cid + nclusters, ...
+    const int tstep = S > 1 ? (1 << 30) : nclusters;
     const int nkb = p.nkb;
     const int kb0 = static_cast<int>(static_cast<int64_t>(rank) * nkb / S);
     const int kb1 = static_cast<int>(static_cast<int64_t>(rank + 1) * nkb / S);
@@ -97,34 +153,28 @@ fp8_gemm_swapab_kernel(const __grid_constant__ Params p, const __grid_constant__
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* ring = smem;
-    uint64_t* full = reinterpret_cast<uint64_t*>(ring + STAGES * C::kStageBytes);
+    uint8_t* aux = ring + STAGES * C::kStageBytes;  // receive area (split) / bf16 staging (unsplit)
+    float* sring = reinterpret_cast<float*>(aux + C::kAuxBytes);
+    uint64_t* full = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(sring) + C::kScaleBytes);
     uint64_t* empty = full + STAGES;
     uint64_t* tfull = empty + STAGES;
     uint64_t* tempty = tfull + kNBuf;
     uint64_t* sfull = tempty + kNBuf;
     uint64_t* sempty = sfull + kSmallScaleSlots;
-    uint64_t* done = sempty + kSmallScaleSlots;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+    uint64_t* done = sempty + kSmallScaleSlots;  // one per MMA warp
+    uint64_t* rbar = done + 2;  // the split partials this CTA receives
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(rbar + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-    float* sring = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(full) + 512);
-    float* red = reinterpret_cast<float*>(ring);  // [TN][128] FP32 partial, after the main loop
-    // Scale ring: kSmallScaleSlots slots of TN sa values followed by sb (TN + 4 floats, 16-byte aligned).
+    int* prefix = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(full) + kSmallBarrierBytes);
+    int* counts = prefix + kMaxMaskedGroups + 1;
+    // A split tile's FP32 partial [TN][128] (weight row fastest) goes into the
+    // ring once the main loop is done; CTA r owns activation rows
+    // [r*TN/S, (r+1)*TN/S) of it.
+    float* red = reinterpret_cast<float*>(ring);
+    const int my_j0 = rank * TN / S, my_j1 = (rank + 1) * TN / S;
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-
-    // Stage `stage` <- the weight tile and the activation tile of K block kb.
-    auto issue_stage = [&](int stage, int kb) {
-        uint8_t* st = ring + stage * C::kStageBytes;
-        const uint64_t pol_w = l2_policy_evict_first();  // weights stream through once
-        const uint64_t pol_a = l2_policy_evict_last();   // activations are re-read by every n-block
-        mbar_arrive_expect_tx(full + stage, C::kStageBytes);
-        tma_load_3d(st, &tmB, full + stage, kb * kBK, n0, g, pol_w);
-        if (MODE == kMasked)
-            tma_load_3d(st + C::kTileBBytes, &tmA, full + stage, kb * kBK, m0, g, pol_a);
-        else
-            tma_load_2d(st + C::kTileBBytes, &tmA, full + stage, kb * kBK, m0, pol_a);
-    };
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -140,225 +190,344 @@ fp8_gemm_swapab_kernel(const __grid_constant__ Params p, const __grid_constant__
             mbar_init(sempty + s, kSmallEpiWarps);
         }
         mbar_init(done, 1);
+        mbar_init(done + 1, 1);
+        mbar_init(rbar, 1);
+        // The whole receive area arrives in one phase: S - 1 slices of this
+        // CTA's rows from the other CTAs of the cluster.
+        if (S > 1) mbar_arrive_expect_tx(rbar, static_cast<uint32_t>((S - 1) * (my_j1 - my_j0) * 128 * 4));
         *abort_flag = 0;
         fence_mbar_init();
-        // The ring starts empty: pull its first weight tiles into L2 while the
-        // previous kernel may still run, then (once its data is visible)
-        // issue the first loads, so that their latency overlaps the rest of
-        // the set-up.
-        prefetch_tmap(&tmA);
-        prefetch_tmap(&tmB);
-        for (int i = 0; i < STAGES && kb0 + i < kb1; ++i) tma_prefetch_3d(&tmB, (kb0 + i) * kBK, n0, g);
-        griddep_wait();
-        for (int i = 0; i < STAGES && kb0 + i < kb1; ++i) issue_stage(i, kb0 + i);
     }
     if (warp == 1) {
-        tmem_alloc(tmem_slot, kSmallTmemCols);
+        tmem_alloc(tmem_slot, C::kTmemCols);
         tmem_relinquish();
     }
-    griddep_wait();
-    griddep_launch_dependents();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    // Every CTA's receive barrier is initialised before any peer copies into it.
+    if (S > 1) cluster_arrive();
     const uint32_t tmem_base = *tmem_slot;
+    // Nothing above touched global memory: with programmatic dependent launch
+    // all of it overlaps the end of the previous kernel in the stream.
+    griddep_launch_dependents();
+    griddep_wait();
+
+    int tiles;
+    if (MODE == kMasked) {
+        // Tiles per group from the device-resident masked_m (clamped to
+        // [0, M_max] and flagged when outside), then an exclusive prefix.
+        for (int g = threadIdx.x; g < p.G; g += kSmallThreads) {
+            int mm = __ldg(p.masked_m + g);
+            if (mm < 0 || mm > p.M) {
+                if (blockIdx.x == 0) atomicOr(&g_dg_error, 4u);
+                mm = min(max(mm, 0), p.M);
+            }
+            counts[g] = mm;
+            prefix[g + 1] = ((mm + TN - 1) / TN) * p.n_blocks;
+        }
+        __syncthreads();
+        if (warp == 0) {
+            int carry = 0;
+            for (int base = 0; base < p.G; base += 32) {
+                const int i = base + lane;
+                int v = (i < p.G) ? prefix[i + 1] : 0;
+#pragma unroll
+                for (int off = 1; off < 32; off <<= 1) {
+                    const int u = __shfl_up_sync(0xffffffffu, v, off);
+                    if (lane >= off) v += u;
+                }
+                if (i < p.G) prefix[i + 1] = v + carry;
+                carry += __shfl_sync(0xffffffffu, v, 31);
+            }
+            if (lane == 0) prefix[0] = 0;
+        }
+        __syncthreads();
+        tiles = prefix[p.G];
+    } else {
+        tiles = p.m_blocks * p.n_blocks;
+    }
 
     if (warp < kSmallFirstEpiWarp) {
-        regs_dec<56>();
         if (warp == 0) {
             // -------------------------------------------------- producer ----
-            // The first STAGES blocks were issued during set-up.
+            // Weights are read once when a group has one TN-row block; with
+            // more, neighbouring clusters re-read each weight tile from L2.
+            const uint64_t pol_w = p.b_stream ? l2_policy_evict_first() : l2_policy_evict_normal();
+            const uint64_t pol_a = l2_policy_evict_last();  // activations are re-read by every n-block
             int stage = 0, fills = 0;
             uint32_t phase = 0;
-            for (int kb = kb0; kb < kb1; ++kb) {
-                if (fills >= STAGES) {
-                    if (!mbar_wait(empty + stage, phase ^ 1u, abort_flag)) break;
-                    if (lane == 0) issue_stage(stage, kb);
+            bool ok = true;
+            for (int t = cid; ok && t < tiles; t += tstep) {
+                const SmallTile tl = small_tile<TN, MODE>(p, t, prefix, counts);
+                for (int kb = kb0; kb < kb1; ++kb) {
+                    if (!mbar_wait(empty + stage, phase ^ 1u, abort_flag)) { ok = false; break; }
+                    if (lane == 0) {
+                        uint8_t* st = ring + stage * C::kStageBytes;
+                        mbar_arrive_expect_tx(full + stage, C::kStageBytes);
+                        tma_load_3d(st, &tmB, full + stage, kb * kBK, tl.n0, tl.g, pol_w);
+                        if (MODE == kMasked)
+                            tma_load_3d(st + C::kTileBBytes, &tmA, full + stage, kb * kBK, tl.m0, tl.g, pol_a);
+                        else
+                            tma_load_2d(st + C::kTileBBytes, &tmA, full + stage, kb * kBK, tl.m0, pol_a);
+                    }
                     __syncwarp();
+                    ++fills;
+                    if (++stage == STAGES) { stage = 0; phase ^= 1u; }
                 }
-                ++fills;
-                if (++stage == STAGES) { stage = 0; phase ^= 1u; }
             }
+            // No copy into this CTA's shared memory may still be in flight
+            // when it exits (matters only after an abort).
             if (lane == 0) {
                 const int first = fills > STAGES ? fills - STAGES : 0;
                 for (int i = first; i < fills; ++i)
                     mbar_wait_drain(full + (i % STAGES), static_cast<uint32_t>((i / STAGES) & 1));
             }
             __syncwarp();
-        } else if (warp == 1) {
+        } else if (warp == 1 || warp == 3) {
             // ------------------------------------------------------- MMA ----
+            // Two warps take alternate K blocks (the CTA's i-th K block goes
+            // to warp 1 for even i, to warp 3 for odd i): issuing four
+            // tcgen05.mma and two commits costs a warp several hundred
+            // cycles, more than the tensor core needs for a 128 x TN x 128
+            // block.  Each block has its own stage and TMEM buffer, so the
+            // two instruction streams never touch the same data.
             constexpr uint32_t idesc = idesc_e4m3_f32(128, TN);
-            int stage = 0, buf = 0;
-            uint32_t phase = 0, bphase = 0;
-            for (int kb = kb0; kb < kb1; ++kb) {
-                if (!mbar_wait(tempty + buf, bphase ^ 1u, abort_flag)) break;
-                if (!mbar_wait(full + stage, phase, abort_flag)) break;
-                tc_fence_after();
-                if (lane == 0) {
-                    const uint32_t w_addr = smem_u32(ring + stage * C::kStageBytes);
-                    const uint32_t a_addr = w_addr + C::kTileBBytes;
-                    const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * TN);
+            const int mw = warp == 1 ? 0 : 1;
+            int i = 0;  // K blocks of this CTA so far, over all its tiles
+            bool ok = true;
+            for (int t = cid; ok && t < tiles; t += tstep) {
+                for (int kb = kb0; kb < kb1; ++kb, ++i) {
+                    if ((i & 1) != mw) continue;
+                    const int stage = i % STAGES, buf = i % kNBuf;
+                    const uint32_t phase = static_cast<uint32_t>(i / STAGES) & 1u;
+                    const uint32_t bphase = static_cast<uint32_t>(i / kNBuf) & 1u;
+                    if (!mbar_wait(tempty + buf, bphase ^ 1u, abort_flag)) { ok = false; break; }
+                    if (!mbar_wait(full + stage, phase, abort_flag)) { ok = false; break; }
+                    tc_fence_after();
+                    if (lane == 0) {
+                        const uint32_t w_addr = smem_u32(ring + stage * C::kStageBytes);
+                        const uint32_t a_addr = w_addr + C::kTileBBytes;
+                        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * TN);
 #pragma unroll
-                    for (int k = 0; k < kBK / 32; ++k)
-                        umma_f8(d_tmem, sdesc_kmajor_sw128(w_addr + k * 32), sdesc_kmajor_sw128(a_addr + k * 32),
-                                idesc, k > 0 ? 1u : 0u);
-                    umma_commit(empty + stage);
-                    umma_commit(tfull + buf);
+                        for (int k = 0; k < kBK / 32; ++k)
+                            umma_f8(d_tmem, sdesc_kmajor_sw128(w_addr + k * 32), sdesc_kmajor_sw128(a_addr + k * 32),
+                                    idesc, k > 0 ? 1u : 0u);
+                        umma_commit(empty + stage);
+                        umma_commit(tfull + buf);
+                    }
+                    __syncwarp();
                 }
-                __syncwarp();
-                if (++stage == STAGES) { stage = 0; phase ^= 1u; }
-                if (++buf == kNBuf) { buf = 0; bphase ^= 1u; }
             }
             if (lane == 0) {
-                umma_commit(done);
-                mbar_wait_drain(done, 0);
+                umma_commit(done + mw);
+                mbar_wait_drain(done + mw, 0);
             }
             __syncwarp();
         } else if (warp == 2) {
             // ------------------------------------------- scale producer ----
-            // Per K block: sa[m0 .. m0+TN) (lane l copies TN/32 consecutive
-            // rows) and sb[n0/128] (lane 0), copied asynchronously.  Up to
-            // kSmallScaleGroup consecutive K blocks share a ring slot whose
-            // barrier completes when all of their copies land.  Rows past the
-            // data are zero-filled and never read.
+            // Per K block: sa of the tile's TN rows (lane l copies TN/32
+            // consecutive rows) and sb of its 128-row weight block (lane 0),
+            // copied asynchronously.  Up to kSmallScaleGroup consecutive K
+            // blocks share a ring slot whose barrier completes when all of
+            // their copies land.  Rows past the data are zero-filled and never
+            // stored.
             constexpr int kPer = TN / 32;  // floats per lane
-            const float* sa_base = p.sa + (MODE == kMasked ? static_cast<int64_t>(g) * nkb * p.sa_stride : 0);
-            const float* sb_row = p.sb + (static_cast<int64_t>(g) * p.nbn + n0 / 128) * nkb;
-            const int r = m0 + lane * kPer;
-            const int left = p.M - r;
-            const uint32_t sa_bytes = left >= kPer ? 4u * kPer : (left > 0 ? 4u * static_cast<uint32_t>(left) : 0u);
             int slot = 0;
             uint32_t sphase = 0;
-            for (int kg = kb0; kg < kb1; kg += kSmallScaleGroup) {
-                if (!mbar_wait(sempty + slot, sphase ^ 1u, abort_flag)) break;
-                const int n = min(kSmallScaleGroup, kb1 - kg);
-                for (int j = 0; j < n; ++j) {
-                    const int kb = kg + j;
-                    const uint32_t dst = smem_u32(sring + (slot * kSmallScaleGroup + j) * (TN + 4));
-                    const float* src = sa_bytes ? sa_base + static_cast<int64_t>(kb) * p.sa_stride + r : p.sa;
-                    if (kPer == 4)
-                        cp_async_16(dst + lane * 16, src, sa_bytes);
-                    else if (kPer == 2)
-                        cp_async_8(dst + lane * 8, src, sa_bytes);
-                    else
-                        cp_async_4(dst + lane * 4, src, sa_bytes);
-                    if (lane == 0) cp_async_4(dst + TN * 4, sb_row + kb, 4u);
+            bool ok = true;
+            for (int t = cid; ok && t < tiles; t += tstep) {
+                const SmallTile tl = small_tile<TN, MODE>(p, t, prefix, counts);
+                const float* sa_base = p.sa + (MODE == kMasked ? static_cast<int64_t>(tl.g) * nkb * p.sa_stride : 0);
+                const float* sb_row = p.sb + (static_cast<int64_t>(tl.g) * p.nbn + tl.n0 / 128) * nkb;
+                const int r = tl.m0 + lane * kPer;
+                const int left = p.M - r;
+                const uint32_t sa_bytes =
+                    left >= kPer ? 4u * kPer : (left > 0 ? 4u * static_cast<uint32_t>(left) : 0u);
+                for (int kg = kb0; kg < kb1; kg += kSmallScaleGroup) {
+                    if (!mbar_wait(sempty + slot, sphase ^ 1u, abort_flag)) { ok = false; break; }
+                    const int n = min(kSmallScaleGroup, kb1 - kg);
+                    for (int j = 0; j < n; ++j) {
+                        const int kb = kg + j;
+                        const uint32_t dst = smem_u32(sring + (slot * kSmallScaleGroup + j) * (TN + 4));
+                        const float* src = sa_bytes ? sa_base + static_cast<int64_t>(kb) * p.sa_stride + r : p.sa;
+                        if (kPer == 4)
+                            cp_async_16(dst + lane * 16, src, sa_bytes);
+                        else if (kPer == 2)
+                            cp_async_8(dst + lane * 8, src, sa_bytes);
+                        else
+                            cp_async_4(dst + lane * 4, src, sa_bytes);
+                        if (lane == 0) cp_async_4(dst + TN * 4, sb_row + kb, 4u);
+                    }
+                    cp_async_arrive(sfull + slot);
+                    if (++slot == kSmallScaleGroups) { slot = 0; sphase ^= 1u; }
                 }
-                cp_async_arrive(sfull + slot);
-                if (++slot == kSmallScaleGroups) { slot = 0; sphase ^= 1u; }
             }
             asm volatile("cp.async.wait_all;" ::: "memory");
         }
+        if (S > 1) {
+            // These warps take part in the cluster barriers only.
+            cluster_wait();
+            cluster_arrive();
+        }
     } else {
         // ------------------------------------------------------ promotion ----
-        regs_inc<192>();
-        float2 acc[TN / 2];
-#pragma unroll
-        for (int j = 0; j < TN / 2; ++j) acc[j] = make_float2(0.f, 0.f);
+        // Warpgroup h promotes activation rows [h*TN/2, (h+1)*TN/2) of every
+        // K block; its four warps cover the 128 weight rows (TMEM lane
+        // quarter = warp % 4).
+        const int ew = warp - kSmallFirstEpiWarp;
+        const int half = ew >> 2;
         const int quarter = warp & 3;
+        const int n = quarter * 32 + lane;              // weight row inside the tile
+        const int j_base = half * C::kCols;
+        const int ptid = threadIdx.x - kSmallFirstEpiWarp * 32;  // 0..255
         const uint32_t t_lane = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16);
         int buf = 0, slot = 0;
         uint32_t bphase = 0, sphase = 0;
-        for (int kb = kb0; kb < kb1; ++kb) {
-            const int jg = (kb - kb0) % kSmallScaleGroup;  // K block inside its scale group
-            if (jg == 0 && !mbar_wait(sfull + slot, sphase, abort_flag)) break;
-            if (!mbar_wait(tfull + buf, bphase, abort_flag)) break;
-            tc_fence_after();
-            // Scales of this K block: s[j] = sa[m0 + j] * sb, formed here.
-            const float* slot_f = sring + (slot * kSmallScaleGroup + jg) * (TN + 4);
-            const float2* sc = reinterpret_cast<const float2*>(slot_f);
-            const float s_b = slot_f[TN];
-            const float2 sb2 = make_float2(s_b, s_b);
+        bool ok = true;
+        float2 acc[C::kCols / 2];
+        for (int t = cid; t < tiles; t += tstep) {
+            const SmallTile tl = small_tile<TN, MODE>(p, t, prefix, counts);
 #pragma unroll
-            for (int cb = 0; cb < C::kChunks; cb += C::kBatch) {
-                uint32_t v[C::kBatch][32];
+            for (int q = 0; q < C::kCols / 2; ++q) acc[q] = make_float2(0.f, 0.f);
+            for (int kb = kb0; ok && kb < kb1; ++kb) {
+                const int jg = (kb - kb0) % kSmallScaleGroup;  // K block inside its scale group
+                if (jg == 0 && !mbar_wait(sfull + slot, sphase, abort_flag)) { ok = false; break; }
+                if (!mbar_wait(tfull + buf, bphase, abort_flag)) { ok = false; break; }
+                tc_fence_after();
+                uint32_t v[C::kChunks][C::kChunk];
 #pragma unroll
-                for (int c = 0; c < C::kBatch; ++c)
-                    tmem_ld_32x32b_x32(t_lane + static_cast<uint32_t>(buf * TN + (cb + c) * 32), v[c]);
+                for (int c = 0; c < C::kChunks; ++c) {
+                    const uint32_t ta = t_lane + static_cast<uint32_t>(buf * TN + j_base + c * C::kChunk);
+                    if constexpr (C::kChunk == 32)
+                        tmem_ld_32x32b_x32(ta, reinterpret_cast<uint32_t(&)[32]>(v[c]));
+                    else
+                        tmem_ld_32x32b_x16(ta, reinterpret_cast<uint32_t(&)[16]>(v[c]));
+                }
                 tmem_ld_wait();
 #pragma unroll
-                for (int c = 0; c < C::kBatch; ++c) reg_fence(v[c]);
-                if (cb + C::kBatch == C::kChunks) {
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(tempty + buf);
-                }
+                for (int c = 0; c < C::kChunks; ++c) reg_fence(v[c]);
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(tempty + buf);
+                // Scales of this K block: s[j] = sa[m0 + j] * sb, formed here.
+                const float* slot_f = sring + (slot * kSmallScaleGroup + jg) * (TN + 4);
+                const float2* sc = reinterpret_cast<const float2*>(slot_f + j_base);
+                const float s_b = slot_f[TN];
+                const float2 sb2 = make_float2(s_b, s_b);
 #pragma unroll
-                for (int c = 0; c < C::kBatch; ++c)
+                for (int c = 0; c < C::kChunks; ++c)
 #pragma unroll
-                    for (int j = 0; j < 16; ++j) {
+                    for (int j = 0; j < C::kChunk / 2; ++j) {
                         const float2 pv = make_float2(__uint_as_float(v[c][2 * j]), __uint_as_float(v[c][2 * j + 1]));
-                        const int q = (cb + c) * 16 + j;
+                        const int q = c * (C::kChunk / 2) + j;
                         acc[q] = __ffma2_rn(pv, __fmul2_rn(sc[q], sb2), acc[q]);
                     }
+                if (jg == kSmallScaleGroup - 1 || kb == kb1 - 1) {
+                    // The group's last K block is done with its scales: release the slot.
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(sempty + slot);
+                    if (++slot == kSmallScaleGroups) { slot = 0; sphase ^= 1u; }
+                }
+                if (++buf == kNBuf) { buf = 0; bphase ^= 1u; }
             }
-            if (jg == kSmallScaleGroup - 1 || kb == kb1 - 1) {
-                // The group's last K block is done with its scales: release the slot.
-                __syncwarp();
-                if (lane == 0) mbar_arrive(sempty + slot);
-                if (++slot == kSmallScaleGroups) { slot = 0; sphase ^= 1u; }
-            }
-            if (++buf == kNBuf) { buf = 0; bphase ^= 1u; }
-        }
-        // The ring is idle once this CTA's last partial has been read out of
-        // TMEM (every load was consumed by an MMA that has completed): it
-        // becomes this CTA's FP32 partial tile red[j][n] (n contiguous).
-        const int n = quarter * 32 + lane;
+            const int64_t d_base = (MODE == kMasked ? static_cast<int64_t>(tl.g) * p.M : 0);
+            if (S == 1) {
+                // ---------------------------- unsplit tile: bf16 store ----
+                // Stage the tile as bf16 [TN][128] (weight row fastest) and
+                // write each row's 128 columns with 16-byte stores.  The first
+                // barrier keeps this tile's staging off the previous tile's
+                // reads.
+                uint16_t* stg = reinterpret_cast<uint16_t*>(aux);
+                named_barrier_sync(1, kSmallEpiThreads);
 #pragma unroll
-        for (int q = 0; q < TN / 2; ++q) {
-            red[(2 * q) * 128 + n] = acc[q].x;
-            red[(2 * q + 1) * 128 + n] = acc[q].y;
+                for (int q = 0; q < C::kCols / 2; ++q) {
+                    const __nv_bfloat162 h = __float22bfloat162_rn(acc[q]);
+                    stg[(j_base + 2 * q) * 128 + n] = *reinterpret_cast<const uint16_t*>(&h.x);
+                    stg[(j_base + 2 * q + 1) * 128 + n] = *reinterpret_cast<const uint16_t*>(&h.y);
+                }
+                named_barrier_sync(1, kSmallEpiThreads);
+                for (int c = ptid; c < TN * 16; c += kSmallEpiThreads) {
+                    const int j = c >> 4, col = tl.n0 + (c & 15) * 8;
+                    const int row = tl.m0 + j;
+                    if (row < tl.rows && col < p.N)
+                        *reinterpret_cast<uint4*>(p.D + (d_base + row) * p.N + col) =
+                            *reinterpret_cast<const uint4*>(stg + j * 128 + (c & 15) * 8);
+                }
+            } else {
+                // ------------------------------ split tile: reduction ----
+                // The ring is idle once this CTA's last partial has been read
+                // out of TMEM (every load was consumed by an MMA that has
+                // completed): it takes the FP32 partial.
+#pragma unroll
+                for (int q = 0; q < C::kCols / 2; ++q) {
+                    red[(j_base + 2 * q) * 128 + n] = acc[q].x;
+                    red[(j_base + 2 * q + 1) * 128 + n] = acc[q].y;
+                }
+                fence_proxy_async_smem();
+                named_barrier_sync(1, kSmallEpiThreads);
+                cluster_wait();  // every peer's receive barrier is initialised
+                if (ptid == 0) {
+                    for (int r = 0; r < S; ++r) {
+                        if (r == rank) continue;
+                        const int j0 = r * TN / S, j1 = (r + 1) * TN / S;
+                        const uint32_t bytes = static_cast<uint32_t>((j1 - j0) * 128 * 4);
+                        const int slot_in_r = rank < r ? rank : rank - 1;
+                        bulk_copy_to_peer(dsmem_addr(smem_u32(aux) + static_cast<uint32_t>(slot_in_r) * bytes, r),
+                                          red + j0 * 128, bytes, dsmem_addr(smem_u32(rbar), r));
+                    }
+                }
+                // This CTA's rows: its own partial plus S - 1 received slices,
+                // added in rank order.
+                if (!mbar_wait(rbar, 0, abort_flag)) {
+                    // Another role gave up: still let copies already on their
+                    // way into this CTA land before it can exit.
+                    ok = false;
+                    mbar_wait_drain(rbar, 0);
+                }
+                const float* rcv = reinterpret_cast<const float*>(aux);
+                const int rows_mine = my_j1 - my_j0;
+                for (int e = ptid; e < rows_mine * 32; e += kSmallEpiThreads) {
+                    const int jj = e >> 5, c4 = (e & 31) * 4;
+                    float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
+                    for (int r = 0; r < S; ++r) {
+                        const float* src = r == rank ? red + (my_j0 + jj) * 128 + c4
+                                                     : rcv + ((r < rank ? r : r - 1) * rows_mine + jj) * 128 + c4;
+                        const float4 v4 = *reinterpret_cast<const float4*>(src);
+                        if (r == 0) {
+                            sum = v4;
+                        } else {
+                            sum.x += v4.x; sum.y += v4.y; sum.z += v4.z; sum.w += v4.w;
+                        }
+                    }
+                    const int row = tl.m0 + my_j0 + jj, col = tl.n0 + c4;
+                    if (row < tl.rows && col < p.N) {
+                        __nv_bfloat162 h0 = __floats2bfloat162_rn(sum.x, sum.y);
+                        __nv_bfloat162 h1 = __floats2bfloat162_rn(sum.z, sum.w);
+                        uint2 pk;
+                        pk.x = *reinterpret_cast<uint32_t*>(&h0);
+                        pk.y = *reinterpret_cast<uint32_t*>(&h1);
+                        *reinterpret_cast<uint2*>(p.D + (d_base + row) * p.N + col) = pk;
+                    }
+                }
+                // Every CTA's receive area is complete past this barrier, so no
+                // bulk copy still reads this CTA's partial.
+                cluster_arrive();
+            }
+        }
+        if (S > 1 && tiles <= cid) {
+            // A cluster without a tile still completes both cluster barriers.
+            cluster_wait();
+            cluster_arrive();
         }
     }
 
-    // -------------------------------------------- split-K reduction ----
-    // CTA `rank` owns float4 groups [rank*E/S, (rank+1)*E/S) of the tile and
-    // adds the S partials in rank order (all loads first, then the sums).
-    constexpr int E4 = TN * 128 / 4;
-    const int e_begin = static_cast<int>(static_cast<int64_t>(rank) * E4 / S);
-    const int e_end = static_cast<int>(static_cast<int64_t>(rank + 1) * E4 / S);
-    const uint32_t red_local = smem_u32(red);
-    auto store4 = [&](int e, float4 sum) {
-        const int j = (e * 4) / 128;
-        const int nn = (e * 4) % 128;
-        const int row = m0 + j, col = n0 + nn;
-        if (row < rows_valid && col < p.N) {
-            const int64_t d_row = (MODE == kMasked ? static_cast<int64_t>(g) * p.M : 0) + row;
-            __nv_bfloat162 h0 = __floats2bfloat162_rn(sum.x, sum.y);
-            __nv_bfloat162 h1 = __floats2bfloat162_rn(sum.z, sum.w);
-            uint2 pk;
-            pk.x = *reinterpret_cast<uint32_t*>(&h0);
-            pk.y = *reinterpret_cast<uint32_t*>(&h1);
-            *reinterpret_cast<uint2*>(p.D + d_row * p.N + col) = pk;
-        }
-    };
-    if (S == 1) {
-        __syncthreads();
-        for (int e = static_cast<int>(threadIdx.x); e < E4; e += kSmallThreads)
-            store4(e, reinterpret_cast<const float4*>(red)[e]);
-    } else {
-        cluster_sync();  // every partial tile written and visible cluster-wide
-        for (int e = e_begin + static_cast<int>(threadIdx.x); e < e_end; e += kSmallThreads) {
-            float4 v[kSmallMaxSplit];
-#pragma unroll
-            for (int r = 0; r < kSmallMaxSplit; ++r)
-                if (r < S) v[r] = ld_dsmem_f4(dsmem_addr(red_local + e * 16, r));
-            float4 sum = v[0];
-#pragma unroll
-            for (int r = 1; r < kSmallMaxSplit; ++r)
-                if (r < S) {
-                    sum.x += v[r].x; sum.y += v[r].y; sum.z += v[r].z; sum.w += v[r].w;
-                }
-            store4(e, sum);
-        }
-        // No CTA may leave while others still read its partial tile.
-        cluster_sync_relaxed();
-    }
+    if (S > 1) cluster_wait();
     tc_fence_before();
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem_base, kSmallTmemCols);
+        tmem_dealloc(tmem_base, C::kTmemCols);
     }
 }
 

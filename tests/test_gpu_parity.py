@@ -266,15 +266,16 @@ def test_masked_under_cuda_graph_follows_device_counts(dgm):
 @pytest.mark.parametrize("M", [1, 17, 32, 33, 64, 100, 128])
 @pytest.mark.parametrize("sms", [148, 16, 3])
 def test_few_rows_split_k_variants(dgm, M, sms):
-    # 35 K blocks: split in 3 or 4 slices of 8-12 blocks on 148 and 16 SMs,
-    # one slice on 3 SMs.
+    # 35 K blocks, 5 weight tiles: clusters of 7 on 148 SMs (TN = 32 or 64),
+    # of 2 on 16 SMs for M <= 64, unsplit where the tiles fill the SMs.
     N, K = 520, 4480
     c = wl.dense_case(M, N, K, seed=M * 3 + sms)
     try:
         dgm.dg_set_num_sms(sms)
         plan = dgm.dg_make_plan(0, M, N, K, 1, sms)
         assert plan["swap_ab"] == 1
-        assert plan["split_k"] == 1 if sms == 3 else plan["split_k"] >= 3
+        want = {148: 7, 16: 2 if M <= 64 else 1, 3: 1}[sms]
+        assert plan["split_k"] == want, plan
         got = run_dense(dgm, c)
     finally:
         dgm.dg_set_num_sms(0)
@@ -282,10 +283,12 @@ def test_few_rows_split_k_variants(dgm, M, sms):
     assert_close(got, ref, mag, f"few rows M={M} split={plan['split_k']}")
 
 
-@pytest.mark.parametrize("K,split", [(1024, 1), (2048, 2), (3072, 3), (3968, 3)])
+@pytest.mark.parametrize("K,split", [(512, 1), (1024, 1), (2048, 4), (3072, 6), (3968, 6)])
 def test_few_rows_split_count_follows_k(dgm, K, split):
-    # Slices keep at least 8 K blocks: 8, 16, 24 and 31 blocks give 1, 2, 3
-    # and 3 slices (31 = 10 + 10 + 11).
+    # 17 weight tiles: below 16 K blocks the split does not repay its
+    # reduction; above, at most 6 CTAs per cluster keep all 17 clusters
+    # resident: 16, 24 and 31 blocks give 4, 6 and 6 slices (31 = 5 + 5 + 5 +
+    # 5 + 5 + 6).
     c = wl.dense_case(64, 2112, K, seed=K)
     assert dgm.dg_make_plan(0, 64, 2112, K, 1, 148)["split_k"] == split
     got = run_dense(dgm, c)
@@ -294,50 +297,32 @@ def test_few_rows_split_count_follows_k(dgm, K, split):
 
 
 def test_few_rows_k_split_uneven(dgm):
-    # 35 K blocks over a cluster of 4 CTAs: slices of 8 and 9 blocks, and the
-    # fixed-order sum must still match.
+    # 35 K blocks over a cluster of 6 CTAs (slices of 5 and 6 blocks) and
+    # 64 activation rows in slices of 10 and 11 rows per CTA: the fixed-order
+    # sum must still match, and repeat bit for bit.
     c = wl.dense_case(64, 2112, 4480, seed=21)
+    assert dgm.dg_make_plan(0, 64, 2112, 4480, 1, 148)["split_k"] == 6
     got = run_dense(dgm, c)
+    assert np.array_equal(run_dense(dgm, c), got)
     ref, mag = oracle_dense(c)
     assert_close(got, ref, mag, "uneven split")
-    assert dgm.dg_make_plan(0, 64, 2112, 4480, 1, 148)["split_k"] == 4
 
 
-# ------------------------------------------- CTA-pair kernel (opt-in path) --
-
-@pytest.fixture
-def force_pair(monkeypatch):
-    monkeypatch.setenv("DG_FORCE_PAIR", "1")
-    yield
-
-
-@pytest.mark.parametrize("M,N,K", [(256, 256, 128), (300, 520, 640), (513, 264, 1024), (129, 136, 256)])
-def test_pair_kernel_dense_full(dgm, force_pair, M, N, K):
-    assert dgm.dg_make_plan(0, M, N, K, 1, 148)["cta_pair"] == 1
-    c = wl.dense_case(M, N, K, seed=M + N + K + 1)
-    got = run_dense(dgm, c)
-    ref, mag = oracle_dense(c)
-    assert_close(got, ref, mag, f"pair dense {M}x{N}x{K}")
-
-
-def test_pair_kernel_dense_large_sampled(dgm, force_pair):
-    c = wl.dense_case(4096, 7168, 2048, seed=0, device="cuda").to("cpu")
-    got = run_dense(dgm, c)
-    rows = sample_rows(4096, seed=8, extra=(255, 256, 383, 384))
+@pytest.mark.parametrize("M,N,K,sms", [(64, 24576, 1536, 148), (128, 4224, 1024, 20), (7, 1040, 512, 3)])
+def test_few_rows_persistent_tiles(dgm, M, N, K, sms):
+    # More weight tiles than SMs: single-CTA clusters walk several tiles each
+    # with one operand ring across them.
+    c = wl.dense_case(M, N, K, seed=M + N + sms)
+    try:
+        dgm.dg_set_num_sms(sms)
+        plan = dgm.dg_make_plan(0, M, N, K, 1, sms)
+        assert plan["split_k"] == 1 and plan["tiles"] > plan["grid"] == sms
+        rows = sample_rows(M, n_random=8, seed=2)
+        got = run_dense(dgm, c)
+    finally:
+        dgm.dg_set_num_sms(0)
     ref, mag = oracle_dense(c, rows=rows)
-    assert_close(got[rows], ref[rows], mag[rows], "pair dense 4096x7168x2048")
-
-
-def test_pair_kernel_masked_full(dgm, force_pair):
-    mm = [300, 0, 257, 1]
-    c = wl.masked_case(4, 300, 264, 512, masked_m=mm, seed=31)
-    assert dgm.dg_make_plan(2, 300, 264, 512, 4, 148)["cta_pair"] == 1
-    got = run_masked(dgm, c)
-    check_masked_untouched(got, mm)
-    ref, mag = oracle_masked(c)
-    for g in range(4):
-        assert_close(got[g, :mm[g]], ref[g, :mm[g]], mag[g, :mm[g]], f"pair masked g={g}")
-    assert dgm.dg_get_device_error() == 0
+    assert_close(got[rows], ref[rows], mag[rows], f"persistent few rows {M}x{N}x{K} on {sms} SMs")
 
 
 # ------------------------------------------- K-split of the last partial wave --
@@ -387,7 +372,8 @@ def test_tail_split_workspaces_stay_bounded_over_many_streams(dgm):
 
 
 # ------------------------------------- back-to-back launches (PDL) --------
-# With DG_PDL=1 GEMM launches allow programmatic dependent launch: a kernel may
+# With PDL on (the default; DG_PDL=0 turns it off) GEMM launches allow
+# programmatic dependent launch: a kernel may
 # start its set-up while the previous kernel in the stream finishes.  It must
 # still read the inputs that kernel wrote, write D after it, and use the
 # K-split workspace only after it.  Each test runs with PDL on and off.

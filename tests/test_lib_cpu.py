@@ -86,13 +86,17 @@ def test_plan_is_consistent(mode, rows, N, K, G):
     assert p["tiles"] == mb * p["n_blocks"]
     assert p["stages"] >= 2
     if p["swap_ab"]:
-        # Few-row kernel: 128 weight rows per tile, one cluster of split_k CTAs
-        # per tile, two CTAs per SM.
+        # Few-row kernel: 128 weight rows per tile, one CTA per SM; K split
+        # over a cluster of split_k CTAs per tile only when the tiles do not
+        # fill the SMs, else single CTAs walk the tiles.
         assert rows <= (256 if mode == 2 else 128)
         assert p["block_n"] == 128 and p["block_m"] in (32, 64, 128)
-        assert 1 <= p["split_k"] <= max(1, min(4, K // 128 // 8))
-        assert p["grid"] == p["tiles"] * p["split_k"]
-        assert p["smem_bytes"] <= 113 * 1024
+        assert 1 <= p["split_k"] <= 8 and (p["split_k"] == 1 or K // 128 // p["split_k"] >= 4)
+        if p["split_k"] > 1:
+            assert p["grid"] == p["tiles"] * p["split_k"] and p["tiles"] < 148
+        else:
+            assert p["grid"] == min(p["tiles"], 148)
+        assert 113 * 1024 < p["smem_bytes"] <= 227 * 1024
     else:
         assert p["block_m"] == 128 and p["block_n"] in (64, 128, 256)
         assert p["split_k"] == 1
@@ -101,24 +105,24 @@ def test_plan_is_consistent(mode, rows, N, K, G):
 
 
 @pytest.mark.parametrize("M,N,K,tn,split", [
-    (1, 2112, 7168, 32, 4), (32, 2112, 7168, 32, 4),
-    # dense tiles of fewer rows than the call has, where more CTAs pay off
-    (64, 2112, 7168, 32, 4), (128, 2112, 7168, 32, 4), (128, 4096, 7168, 64, 4), (128, 7168, 2048, 64, 2),
-    # enough weight tiles already: the smallest TN that holds the rows
-    (64, 24576, 1536, 64, 1), (128, 24576, 1536, 128, 1), (128, 32768, 512, 128, 1), (128, 7168, 16384, 128, 4),
+    # the planner's cost model (fitted to measured decode timings) on the sweep
+    (1, 2112, 7168, 32, 6), (32, 2112, 7168, 32, 6), (64, 2112, 7168, 64, 6), (128, 2112, 7168, 64, 3),
+    (64, 4096, 7168, 64, 4), (128, 4096, 7168, 128, 4), (64, 7168, 2048, 32, 1), (128, 7168, 2048, 64, 1),
+    (64, 7168, 16384, 64, 2), (128, 7168, 16384, 128, 2),
+    (64, 24576, 1536, 64, 1), (128, 24576, 1536, 128, 1), (64, 32768, 512, 64, 1), (128, 32768, 512, 128, 1),
 ])
 def test_few_row_plan_tile_and_split(M, N, K, tn, split):
     p = dg.dg_make_plan(0, M, N, K, 1, 148)
-    assert p["swap_ab"] == 1 and p["block_m"] == tn and p["split_k"] == split
+    assert p["swap_ab"] == 1 and p["block_m"] == tn and p["split_k"] == split, p
     assert p["m_blocks"] == -(-M // tn) and p["n_blocks"] == -(-N // 128)
     assert dg.dg_make_plan(0, 129, N, K, 1, 148)["swap_ab"] == 0
 
 
-def test_few_row_plan_never_exceeds_the_rows_tile():
+def test_few_row_plan_tile_never_taller_than_the_rows_need():
     for M in range(1, 129):
         p = dg.dg_make_plan(0, M, 520, 4480, 1, 148)
         assert p["block_m"] <= (32 if M <= 32 else 64 if M <= 64 else 128)
-        assert 1 <= p["split_k"] <= 4 and p["grid"] == p["tiles"] * p["split_k"]
+        assert p["m_blocks"] == -(-M // p["block_m"]) and p["grid"] == p["tiles"] * p["split_k"]
 
 
 @pytest.mark.parametrize("args,expect", [
@@ -189,6 +193,8 @@ def test_binding_fails_loudly_when_library_missing(tmp_path, monkeypatch):
 def test_pdl_switch_defaults_to_the_environment(monkeypatch):
     try:
         dg.dg_set_pdl(None)
+        monkeypatch.delenv("DG_PDL", raising=False)
+        assert dg.dg_get_pdl() is True  # on unless DG_PDL=0
         monkeypatch.setenv("DG_PDL", "1")
         assert dg.dg_get_pdl() is True
         monkeypatch.setenv("DG_PDL", "0")

@@ -4,11 +4,11 @@ For random dense, contiguous and masked problems on 1..148 SMs, dg_make_plan
 must return a plan whose tile arithmetic is exact and whose kernel choice
 respects the limits the kernels are built for:
   * few-row problems (dense M <= 128, masked M_max <= 256) take the swap-AB
-    split-K kernel: 128 weight rows per tile, TN in {32, 64, 128} activation
-    rows (masked: the smallest that holds min(M_max, 128); dense: that size or
-    a half / quarter of it, at least 32), 1..4 K slices of at least 8 K blocks
-    (or one slice), one cluster per tile, <= 113 KiB of shared memory so that
-    two CTAs share an SM;
+    kernel: 128 weight rows per tile, TN in {32, 64, 128} activation rows (no
+    taller than min(rows, 128) needs), one CTA per SM; K is split into S
+    slices of at least 4 K blocks only when the tiles do not fill the SMs, with
+    one cluster of S CTAs per tile and every cluster resident at once;
+    otherwise single-CTA clusters walk the tiles (grid = min(tiles, SMs));
   * everything else takes the persistent 128 x BN kernel (BN in {64, 128,
     256}) with at most one CTA per SM, and dense calls may split the tiles of a
     partial last wave into 2..8 K slices of at least 16 K blocks that the idle
@@ -30,6 +30,11 @@ def built_library():
 
 def cdiv(a, b):
     return -(-a // b)
+
+
+# CTAs of one-CTA-per-SM clusters of size S resident at once on a 148-SM B200
+# (cudaOccupancyMaxActiveClusters x S).
+CLUSTER_CAPACITY = {1: 148, 2: 148, 3: 135, 4: 132, 5: 130, 6: 132, 7: 105, 8: 120}
 
 
 def smallest_tn(rows):
@@ -62,19 +67,21 @@ def test_plan_invariants(problem):
     assert p["m_blocks"] == groups * cdiv(rows, p["block_m"])
     assert p["tiles"] == p["m_blocks"] * p["n_blocks"]
     assert p["stages"] >= 2 and p["smem_bytes"] <= 227 * 1024
-    assert p["cta_pair"] == 0  # CTA pairs are opt-in only
     few_rows = (mode == 0 and rows <= 128) or (mode == 2 and rows <= 256)
     assert p["swap_ab"] == int(few_rows)
     if few_rows:
         assert p["block_n"] == 128
-        t0 = smallest_tn(min(rows, 128))
-        if mode == 2:
-            assert p["block_m"] == t0
+        assert p["block_m"] in (32, 64, 128) and p["block_m"] <= smallest_tn(min(rows, 128))
+        S = p["split_k"]
+        assert 1 <= S <= (4 if p["block_m"] == 128 else 8)
+        if S > 1:
+            # split only when the tiles do not fill the SMs, slices of >= 4
+            # K blocks, one cluster per tile, all clusters resident at once
+            assert p["tiles"] < sms and nkb // S >= 4
+            assert p["grid"] == p["tiles"] * S <= CLUSTER_CAPACITY[S] * sms // 148
         else:
-            assert p["block_m"] in (t0, t0 // 2, t0 // 4) and p["block_m"] >= 32
-        assert 1 <= p["split_k"] <= max(1, min(4, nkb // 8))
-        assert p["grid"] == p["tiles"] * p["split_k"]
-        assert p["smem_bytes"] <= 113 * 1024
+            assert p["grid"] == min(p["tiles"], sms)
+        assert p["smem_bytes"] > 113 * 1024  # one CTA per SM
         assert p["tail_split"] == 1
     else:
         assert p["block_m"] == 128 and p["block_n"] in (64, 128, 256)
@@ -89,7 +96,10 @@ def test_plan_invariants(problem):
             assert S == 1
 
 
-def test_few_row_split_grows_with_k_until_four_slices():
-    # One weight tile (N = 128), so SMs never cap the split: the K-block count does.
+def test_few_row_split_grows_with_k_until_the_cluster_cap():
+    # One weight tile (N = 128), so SMs never cap the split: the K-block count
+    # (slices of >= 4 blocks, and long enough to repay the reduction) and the
+    # cluster size cap (8 for TN <= 64) do.
     got = [dg.dg_make_plan(0, 64, 128, 128 * nkb, 1, 148)["split_k"] for nkb in (4, 8, 15, 16, 24, 32, 64, 256)]
-    assert got == [1, 1, 1, 2, 3, 4, 4, 4]
+    assert got == [1, 1, 3, 4, 6, 8, 8, 8]
+    assert all(a <= b for a, b in zip(got, got[1:]))
