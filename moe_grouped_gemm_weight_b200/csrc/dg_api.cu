@@ -206,6 +206,13 @@ Choice choose(int m_blocks, int N, int num_sms, bool mn_major = false) {
     return best;
 }
 
+// Dense NT calls of 128 x 256 tiles with at most kShortKBlocks K blocks per
+// tile stage each promotion warp's whole epilogue at once (a 3-stage ring
+// leaves room): with few K blocks per tile the epilogue is a large share of
+// its time.
+constexpr int kShortKBlocks = 16;
+constexpr int kShortKStages = 3;
+
 int plan_smem(const Choice& c) {
     return c.bn == 256 ? smem_for<256>() : c.bn == 128 ? smem_for<128>() : smem_for<64>();
 }
@@ -368,6 +375,10 @@ dg_status plan(int mode, int rows, int N, int K, int G, int num_sms, dg_plan* ou
     out->tiles = m_blocks * out->n_blocks;
     out->grid = (mode == 2) ? num_sms : (out->tiles < num_sms ? out->tiles : num_sms);
     out->smem_bytes = plan_smem(c);
+    if (mode == 0 && layout == 0 && c.bn == 256 && K / dg::kBK <= kShortKBlocks) {
+        out->stages = kShortKStages;
+        out->smem_bytes = dg::smem_bytes<256, kShortKStages, 4>();
+    }
     out->swap_ab = 0;
     out->split_k = 1;
     out->tail_split = 1;
@@ -417,12 +428,12 @@ void set_pdl(cudaLaunchAttribute& a) {
     a.val.programmaticStreamSerializationAllowed = pdl_enabled() ? 1 : 0;
 }
 
-template <int BN, int STAGES, int MODE, int LAYOUT = 0>
+template <int BN, int STAGES, int MODE, int LAYOUT = 0, int SP = 1>
 dg_status launch_one(const dg::Params& p, const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& td,
                      int grid, cudaStream_t stream) {
-    constexpr int smem = dg::smem_bytes<BN, STAGES>();
+    constexpr int smem = dg::smem_bytes<BN, STAGES, SP>();
     static_assert(smem <= 227 * 1024, "shared memory budget exceeded");
-    auto kern = dg::fp8_gemm_kernel<BN, STAGES, MODE, LAYOUT>;
+    auto kern = dg::fp8_gemm_kernel<BN, STAGES, MODE, LAYOUT, SP>;
     static std::atomic<int> attr_set[kMaxDevices];
     int dev = 0;
     cudaGetDevice(&dev);
@@ -493,7 +504,10 @@ template <int MODE>
 dg_status dispatch(const dg_plan& pl, const dg::Params& p, const CUtensorMap& ta, const CUtensorMap& tb,
                    const CUtensorMap& td, cudaStream_t stream) {
     switch (pl.block_n) {
-        case 256: return launch_one<256, max_stages<256>(), MODE>(p, ta, tb, td, pl.grid, stream);
+        case 256:
+            if (MODE == dg::kDense && pl.stages == kShortKStages)
+                return launch_one<256, kShortKStages, MODE, 0, 4>(p, ta, tb, td, pl.grid, stream);
+            return launch_one<256, max_stages<256>(), MODE>(p, ta, tb, td, pl.grid, stream);
         case 128: return launch_one<128, max_stages<128>(), MODE>(p, ta, tb, td, pl.grid, stream);
         case 64: return launch_one<64, max_stages<64>(), MODE>(p, ta, tb, td, pl.grid, stream);
         default: return fail(DG_ERR_UNSUPPORTED, "no kernel for block_n=%d", pl.block_n);

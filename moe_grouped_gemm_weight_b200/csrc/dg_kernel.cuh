@@ -132,11 +132,12 @@ struct Cfg {
     static_assert(kChunks % kBatch == 0, "chunk batching");
 };
 
-template <int BN, int STAGES>
+template <int BN, int STAGES, int SP = 1>
 constexpr int smem_bytes() {
-    // 1 KiB alignment slack + operand ring + output staging + barriers and
-    // bookkeeping (512 B) + scale ring + masked prefix table.
-    return 1024 + STAGES * (kTileABytes + Cfg<BN>::kTileBBytes) + Cfg<BN>::kEpiWarpsC * kStageOutBytes + 512 +
+    // 1 KiB alignment slack + operand ring + output staging (SP pieces of
+    // 32 x 32 bf16 per promotion warp) + barriers and bookkeeping (512 B) +
+    // scale ring + masked prefix table.
+    return 1024 + STAGES * (kTileABytes + Cfg<BN>::kTileBBytes) + Cfg<BN>::kEpiWarpsC * SP * kStageOutBytes + 512 +
            kScaleSlots * kScaleSlotFloats * 4 + 4 * (kMaxMaskedGroups + 1);
 }
 
@@ -222,7 +223,12 @@ __device__ __forceinline__ void group_k_range(const Params& p, const Tile& tl, W
 // [K][M] (M-major, the "T" of TN / TT), bit 1 set = B stored [K][N] (N-major,
 // the "N" of NN / TN); clear = K-major as in NT.  An MN-major operand is loaded
 // as 128 x 128 TMA boxes (MN inner) and described to the MMA as MN-major.
-template <int BN, int STAGES, int MODE, int LAYOUT = 0>
+// SP: staging pieces per promotion warp.  With one, each 32 x 32 piece of
+// the epilogue waits until the previous piece's TMA store has read the
+// buffer; with one per piece of the warp's columns, a tile's whole epilogue
+// is staged and stored without waiting (the next tile's epilogue waits once),
+// which pays on short K where the epilogue is a large share of a tile.
+template <int BN, int STAGES, int MODE, int LAYOUT = 0, int SP = 1>
 __global__ void __launch_bounds__(Cfg<BN>::kThreadsC, 1)
 fp8_gemm_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtensorMap tmA,
                 const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmD) {
@@ -238,8 +244,8 @@ fp8_gemm_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtens
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* sA = smem;
     uint8_t* sB = sA + STAGES * kTileABytes;
-    uint8_t* sOut = sB + STAGES * C::kTileBBytes;  // 1 KiB aligned, kStageOutBytes per promotion warp
-    uint64_t* full = reinterpret_cast<uint64_t*>(sOut + C::kEpiWarpsC * kStageOutBytes);
+    uint8_t* sOut = sB + STAGES * C::kTileBBytes;  // 1 KiB aligned, SP x kStageOutBytes per promotion warp
+    uint64_t* full = reinterpret_cast<uint64_t*>(sOut + C::kEpiWarpsC * SP * kStageOutBytes);
     uint64_t* empty = full + STAGES;
     uint64_t* tfull = empty + STAGES;
     uint64_t* tempty = tfull + kNBuf;
@@ -618,11 +624,19 @@ fp8_gemm_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtens
             // rows, rows past masked_m) store their valid rows directly.
             const bool clip_ok = row_ok || MODE == kDense || MODE == kKGrouped || (MODE == kMasked && row >= p.M);
             if (__all_sync(0xffffffffu, clip_ok)) {
-                const uint32_t stg = smem_u32(sOut + ew * kStageOutBytes);
+                static_assert(SP == 1 || SP == C::kColsPerWarp / 32, "one staging piece, or one per piece");
+                if (SP > 1) {
+                    if (lane == 0) bulk_wait_read<0>();  // the previous tile's stores have read every piece
+                    __syncwarp();
+                }
 #pragma unroll
                 for (int pc = 0; pc < C::kColsPerWarp / 32; ++pc) {
-                    if (lane == 0) bulk_wait_read<0>();  // previous store has read the buffer
-                    __syncwarp();
+                    uint8_t* piece = sOut + (ew * SP + (SP > 1 ? pc : 0)) * kStageOutBytes;
+                    const uint32_t stg = smem_u32(piece);
+                    if (SP == 1) {
+                        if (lane == 0) bulk_wait_read<0>();  // previous store has read the buffer
+                        __syncwarp();
+                    }
 #pragma unroll
                     for (int q = 0; q < 4; ++q) {
                         __nv_bfloat162 h0 = __float22bfloat162_rn(acc[pc * 16 + q * 4 + 0]);
@@ -638,9 +652,9 @@ fp8_gemm_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtens
                     const int x = tl.n0 + col0 + pc * 32;
                     if (lane == 0 && x < p.N) {
                         if (MODE == kMasked || MODE == kKGrouped)
-                            tma_store_3d(&tmD, sOut + ew * kStageOutBytes, x, tl.m0 + quarter * 32, g);
+                            tma_store_3d(&tmD, piece, x, tl.m0 + quarter * 32, g);
                         else
-                            tma_store_2d(&tmD, sOut + ew * kStageOutBytes, x, tl.m0 + quarter * 32);
+                            tma_store_2d(&tmD, piece, x, tl.m0 + quarter * 32);
                         bulk_commit();
                     }
                 }

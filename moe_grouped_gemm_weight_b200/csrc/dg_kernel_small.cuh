@@ -485,21 +485,27 @@ fp8_gemm_swapab_kernel(const __grid_constant__ Params p, const __grid_constant__
                     ok = false;
                     mbar_wait_drain(rbar, 0);
                 }
+                // Everything this CTA receives has landed: arrive now, so the
+                // barrier that keeps each CTA alive until every copy out of it
+                // has completed overlaps the sums below.
+                cluster_arrive();
                 const float* rcv = reinterpret_cast<const float*>(aux);
                 const int rows_mine = my_j1 - my_j0;
                 for (int e = ptid; e < rows_mine * 32; e += kSmallEpiThreads) {
                     const int jj = e >> 5, c4 = (e & 31) * 4;
                     float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
-                    for (int r = 0; r < S; ++r) {
-                        const float* src = r == rank ? red + (my_j0 + jj) * 128 + c4
-                                                     : rcv + ((r < rank ? r : r - 1) * rows_mine + jj) * 128 + c4;
-                        const float4 v4 = *reinterpret_cast<const float4*>(src);
-                        if (r == 0) {
-                            sum = v4;
-                        } else {
-                            sum.x += v4.x; sum.y += v4.y; sum.z += v4.z; sum.w += v4.w;
+#pragma unroll
+                    for (int r = 0; r < C::kMaxSplit; ++r)
+                        if (r < S) {
+                            const float* src = r == rank ? red + (my_j0 + jj) * 128 + c4
+                                                         : rcv + ((r < rank ? r : r - 1) * rows_mine + jj) * 128 + c4;
+                            const float4 v4 = *reinterpret_cast<const float4*>(src);
+                            if (r == 0) {
+                                sum = v4;
+                            } else {
+                                sum.x += v4.x; sum.y += v4.y; sum.z += v4.z; sum.w += v4.w;
+                            }
                         }
-                    }
                     const int row = tl.m0 + my_j0 + jj, col = tl.n0 + c4;
                     if (row < tl.rows && col < p.N) {
                         __nv_bfloat162 h0 = __floats2bfloat162_rn(sum.x, sum.y);
@@ -510,9 +516,6 @@ fp8_gemm_swapab_kernel(const __grid_constant__ Params p, const __grid_constant__
                         *reinterpret_cast<uint2*>(p.D + (d_base + row) * p.N + col) = pk;
                     }
                 }
-                // Every CTA's receive area is complete past this barrier, so no
-                // bulk copy still reads this CTA's partial.
-                cluster_arrive();
             }
         }
         if (S > 1 && tiles <= cid) {
