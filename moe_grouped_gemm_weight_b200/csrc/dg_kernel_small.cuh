@@ -211,6 +211,15 @@ fp8_gemm_swapab_kernel(const __grid_constant__ Params p, const __grid_constant__
     // Nothing above touched global memory: with programmatic dependent launch
     // all of it overlaps the end of the previous kernel in the stream.
     griddep_launch_dependents();
+    if (MODE != kMasked && threadIdx.x == 0 && cid < p.m_blocks * p.n_blocks) {
+        // Pull this CTA's first weight tiles into L2 while the previous kernel
+        // may still run.  L2 is the point of coherence, so a prefetch issued
+        // before the dependency wait never makes a later read return data
+        // older than the wait exposes.  (Masked tiles depend on masked_m,
+        // which the previous kernel may write.)
+        const int n0 = (cid / p.m_blocks) * 128;
+        for (int i = 0; i < STAGES && kb0 + i < kb1; ++i) tma_prefetch_3d(&tmB, (kb0 + i) * kBK, n0, 0);
+    }
     griddep_wait();
 
     int tiles;
@@ -326,12 +335,12 @@ fp8_gemm_swapab_kernel(const __grid_constant__ Params p, const __grid_constant__
             __syncwarp();
         } else if (warp == 2) {
             // ------------------------------------------- scale producer ----
-            // Per K block: sa of the tile's TN rows (lane l copies TN/32
-            // consecutive rows) and sb of its 128-row weight block (lane 0),
-            // copied asynchronously.  Up to kSmallScaleGroup consecutive K
-            // blocks share a ring slot whose barrier completes when all of
-            // their copies land.  Rows past the data are zero-filled and never
-            // stored.
+            // Per K block: the products sa[m0 + j] * sb for the tile's TN
+            // activation rows (lane l forms TN/32 consecutive rows) and its
+            // 128-row weight block, so that promotion is one FMA per value.
+            // Up to kSmallScaleGroup consecutive K blocks share a ring slot
+            // whose barrier completes when all 32 lanes have written theirs.
+            // Rows past the data get zero scales and are never stored.
             constexpr int kPer = TN / 32;  // floats per lane
             int slot = 0;
             uint32_t sphase = 0;
@@ -342,28 +351,30 @@ fp8_gemm_swapab_kernel(const __grid_constant__ Params p, const __grid_constant__
                 const float* sb_row = p.sb + (static_cast<int64_t>(tl.g) * p.nbn + tl.n0 / 128) * nkb;
                 const int r = tl.m0 + lane * kPer;
                 const int left = p.M - r;
-                const uint32_t sa_bytes =
-                    left >= kPer ? 4u * kPer : (left > 0 ? 4u * static_cast<uint32_t>(left) : 0u);
+                const int nvalid = left >= kPer ? kPer : (left > 0 ? left : 0);
                 for (int kg = kb0; kg < kb1; kg += kSmallScaleGroup) {
                     if (!mbar_wait(sempty + slot, sphase ^ 1u, abort_flag)) { ok = false; break; }
                     const int n = min(kSmallScaleGroup, kb1 - kg);
-                    for (int j = 0; j < n; ++j) {
-                        const int kb = kg + j;
-                        const uint32_t dst = smem_u32(sring + (slot * kSmallScaleGroup + j) * (TN + 4));
-                        const float* src = sa_bytes ? sa_base + static_cast<int64_t>(kb) * p.sa_stride + r : p.sa;
-                        if (kPer == 4)
-                            cp_async_16(dst + lane * 16, src, sa_bytes);
-                        else if (kPer == 2)
-                            cp_async_8(dst + lane * 8, src, sa_bytes);
-                        else
-                            cp_async_4(dst + lane * 4, src, sa_bytes);
-                        if (lane == 0) cp_async_4(dst + TN * 4, sb_row + kb, 4u);
+                    float sav[kSmallScaleGroup][kPer];
+                    float sbv[kSmallScaleGroup];
+#pragma unroll
+                    for (int j = 0; j < kSmallScaleGroup; ++j) {
+                        sbv[j] = j < n ? __ldg(sb_row + kg + j) : 0.f;
+#pragma unroll
+                        for (int e = 0; e < kPer; ++e)
+                            sav[j][e] = (j < n && e < nvalid) ? __ldg(sa_base + static_cast<int64_t>(kg + j) * p.sa_stride + r + e) : 0.f;
                     }
-                    cp_async_arrive(sfull + slot);
+#pragma unroll
+                    for (int j = 0; j < kSmallScaleGroup; ++j)
+                        if (j < n) {
+                            float* dstf = sring + (slot * kSmallScaleGroup + j) * (TN + 4);
+#pragma unroll
+                            for (int e = 0; e < kPer; ++e) dstf[lane * kPer + e] = sav[j][e] * sbv[j];
+                        }
+                    mbar_arrive(sfull + slot);
                     if (++slot == kSmallScaleGroups) { slot = 0; sphase ^= 1u; }
                 }
             }
-            asm volatile("cp.async.wait_all;" ::: "memory");
         }
         if (S > 1) {
             // These warps take part in the cluster barriers only.
@@ -410,18 +421,17 @@ fp8_gemm_swapab_kernel(const __grid_constant__ Params p, const __grid_constant__
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(tempty + buf);
-                // Scales of this K block: s[j] = sa[m0 + j] * sb, formed here.
+                // Scales of this K block: s[j] = sa[m0 + j] * sb, formed by the
+                // scale warp.
                 const float* slot_f = sring + (slot * kSmallScaleGroup + jg) * (TN + 4);
                 const float2* sc = reinterpret_cast<const float2*>(slot_f + j_base);
-                const float s_b = slot_f[TN];
-                const float2 sb2 = make_float2(s_b, s_b);
 #pragma unroll
                 for (int c = 0; c < C::kChunks; ++c)
 #pragma unroll
                     for (int j = 0; j < C::kChunk / 2; ++j) {
                         const float2 pv = make_float2(__uint_as_float(v[c][2 * j]), __uint_as_float(v[c][2 * j + 1]));
                         const int q = c * (C::kChunk / 2) + j;
-                        acc[q] = __ffma2_rn(pv, __fmul2_rn(sc[q], sb2), acc[q]);
+                        acc[q] = __ffma2_rn(pv, sc[q], acc[q]);
                     }
                 if (jg == kSmallScaleGroup - 1 || kb == kb1 - 1) {
                     // The group's last K block is done with its scales: release the slot.
