@@ -158,10 +158,13 @@ DG_API dg_status dg_k_grouped_fp8_gemm_tn(uint16_t* D, const uint8_t* A, const f
  * summation order (tolerance as for dg_fp8_gemm_nt).  A scale that is not a
  * power of two sets DG_DEVERR_NOT_POW2 in the device error word and its tile's
  * results are then wrong; the call does not check the scales on the host.
- * The block-scaled kernel is used where it measured faster than the promotion
- * kernel (K <= 2048 with at least two waves of 128 x 256 tiles); other shapes
- * take the promotion kernel (the same result, no DG_DEVERR_NOT_POW2 check).
- * DG_FORCE_BLOCK_SCALED=1 in the environment forces the block-scaled kernel.
+ * The block-scaled kernel is used for M > 256, where it measured faster than
+ * the promotion kernel; fewer rows take the promotion path (the same result,
+ * no DG_DEVERR_NOT_POW2 check).  DG_FORCE_BLOCK_SCALED=1 in the environment
+ * forces the block-scaled kernel, =0 the promotion path.  Like
+ * dg_fp8_gemm_nt, the call may split the tiles of a partial last wave (or all
+ * tiles, when there are fewer than SMs) along K; the split uses the stream's
+ * K-split workspace (see "Workspace" above) and is deterministic.
  */
 DG_API dg_status dg_fp8_gemm_nt_ue8m0(uint16_t* D, const uint8_t* A, const float* sa, int sa_stride,
                                       const uint8_t* B, const float* sb, int M, int N, int K, void* stream);

@@ -903,6 +903,22 @@ dg_status dg_fp8_gemm_nt_noalloc(uint16_t* D, const uint8_t* A, const float* sa,
     return dispatch<dg::kDense>(pl, p, ta, tb, td, st);
 }
 
+// K-split of the block-scaled kernel: the R tiles left after the full waves
+// (all tiles when there are fewer than SMs) are each split into S K slices
+// run by otherwise idle CTAs.  The rule is the promotion kernel's tail split:
+// S ~ sqrt(nkb / 1.5) balances a slice's K blocks against slice 0's
+// reduction of S-1 partials; S*R <= SMs, S <= 8, and at least 16 K blocks
+// per slice.  Returns 1 for no split.
+static int ue8m0_split(int tiles, int nkb, int sms) {
+    const int rest = tiles % sms;
+    if (rest == 0) return 1;
+    int split = static_cast<int>(std::sqrt(nkb / 1.5) + 0.5);
+    if (split > sms / rest) split = sms / rest;
+    if (split > 8) split = 8;
+    if (split > nkb / 16) split = nkb / 16;
+    return split >= 2 ? split : 1;
+}
+
 dg_status dg_fp8_gemm_nt_ue8m0(uint16_t* D, const uint8_t* A, const float* sa, int sa_stride, const uint8_t* B,
                                const float* sb, int M, int N, int K, void* stream) {
     dg_status s = check_sizes(0, M, N, K, 1);
@@ -911,18 +927,19 @@ dg_status dg_fp8_gemm_nt_ue8m0(uint16_t* D, const uint8_t* A, const float* sa, i
     if (M == 0) return ok();
     const int sms = effective_sms();
     if (sms <= 0) return fail(DG_ERR_CUDA, "no CUDA device");
-    // The block-scaled kernel has no K-split tail and a fixed 128 x 256 tile.
-    // Measured against the promotion kernel on power-of-two scales (CUDA-graph
-    // replays on B200) it is faster when K <= 2048 and there are at least two
-    // waves of tiles (4096x32768x512 by 25 %, 4096x24576x1536 by 8 %,
-    // 4096x7168x2048 by 3 %) and slower otherwise (4096x7168x16384 by 20 %,
-    // where the promotion kernel splits the partial last wave).  Elsewhere the
-    // call takes the promotion kernel, which computes the same sum for any
-    // FP32 scales.  DG_FORCE_BLOCK_SCALED=1 always takes the block-scaled one.
+    // Routing.  With the scale-factor conversion split over two warps and the
+    // K-split of a partial last wave, the block-scaled kernel measured faster
+    // than the promotion kernel on power-of-two scales (CUDA-graph replays on
+    // B200) on every M = 4096 shape of the dense sweep, by 4 % (7168 x 16384)
+    // to 25 % (32768 x 512), and 5 % slower at 256 x 7168 x 7168.  So M > 256
+    // takes it; fewer rows go to the promotion path, whose few-row kernel
+    // streams the weights with 32- or 64-row tiles.  DG_FORCE_BLOCK_SCALED=1
+    // always takes the block-scaled kernel, =0 never.
     {
         const char* force = std::getenv("DG_FORCE_BLOCK_SCALED");
-        const int ue_tiles = cdiv(M, dg::kBM) * cdiv(N, dg::kUeBN);
-        const bool block_scaled = (force && force[0] == '1') || (K <= 2048 && ue_tiles >= 2 * sms);
+        bool block_scaled = M > 256;
+        if (force && force[0] == '1') block_scaled = true;
+        if (force && force[0] == '0') block_scaled = false;
         if (!block_scaled) return dg_fp8_gemm_nt(D, A, sa, sa_stride, B, sb, M, N, K, stream);
     }
     dg_plan pl{};
@@ -934,13 +951,21 @@ dg_status dg_fp8_gemm_nt_ue8m0(uint16_t* D, const uint8_t* A, const float* sa, i
     pl.tiles = pl.m_blocks * pl.n_blocks;
     pl.grid = pl.tiles < sms ? pl.tiles : sms;
     pl.split_k = 1;
-    pl.tail_split = 1;
+    pl.tail_split = ue8m0_split(pl.tiles, K / dg::kBK, sms);
+    if (pl.tail_split > 1 && pl.tiles < sms) pl.grid = pl.tiles * pl.tail_split;
     CUtensorMap ta, tb, td;
     if ((s = make_operand_map(&ta, A, K, M, 1, dg::kBM, false)) != DG_OK) return s;
     if ((s = make_operand_map(&tb, B, K, N, 1, dg::kUeBN, true)) != DG_OK) return s;
     if ((s = make_output_map(&td, D, N, M, 1, false)) != DG_OK) return s;
     dg::Params p = make_params(D, sa, sa_stride, sb, M, N, K, 1, pl);
     p.b_stream = pl.m_blocks == 1;
+    TailWorkspace ws;
+    if (pl.tail_split > 1 && tail_workspace(static_cast<cudaStream_t>(stream), &ws)) {
+        p.tail_split = pl.tail_split;
+        p.full_tiles = (pl.tiles / pl.grid) * pl.grid;
+        p.ws = ws.partials;
+        p.ws_flags = ws.flags;
+    }
     constexpr int smem = dg::ue8m0_smem_bytes();
     static_assert(smem <= 227 * 1024, "shared memory budget exceeded");
     auto kern = dg::fp8_gemm_ue8m0_kernel;

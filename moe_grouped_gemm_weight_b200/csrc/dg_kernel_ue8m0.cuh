@@ -18,16 +18,19 @@
 // (section 3.1) notes that on SM100 the scales are UE8M0.  This kernel is the
 // SM100 path for such scales; the general FP32-scale kernels stay the default.
 //
-// Tiles 128 x 256, persistent CTAs of 384 threads:
+// Tiles 128 x 256, persistent CTAs of 384 threads.  The work items are those
+// of the promotion kernel: whole tiles round-robin, and, when the planner asks
+// for it, the tiles of the last partial wave (or all tiles, when there are
+// fewer than CTAs) split into K slices whose FP32 partials slice 0 adds up.
 //   warp 0      TMA producer (A 128x128 and B 256x128 per K block, 4 stages)
 //   warp 1      TMEM owner; per four K blocks copies their scale factors from
 //               shared memory to TMEM (tcgen05.cp); per K block issues 4 MMAs
-//   warp 2      scale loader: sa (128 rows) and sb (2 blocks) per K block by
-//               cp.async into an 8-slot FP32 ring
-//   warp 3      scale converter: FP32 -> UE8M0 codes in the scale-factor
-//               layout, 8-slot ring; a scale that is not a positive normal
-//               power of two sets DG_DEVERR_NOT_POW2 (its code is still its
-//               exponent field, so the result is wrong for it)
+//   warps 2-3   scale converters, taking alternate groups of four K blocks:
+//               FP32 sa (128 rows) and sb (2 blocks) read from global memory,
+//               UE8M0 codes written in the scale-factor layout, 8-slot ring;
+//               a scale that is not a positive normal power of two sets
+//               DG_DEVERR_NOT_POW2 (its code is still its exponent field, so
+//               the result is wrong for it)
 //   warps 4-11  epilogue: TMEM -> bf16 -> TMA store (two warpgroups of 128
 //               columns)
 // Scale-factor layout in shared memory (one 512-byte block per 128 rows or
@@ -51,8 +54,6 @@ constexpr int kUeSfbBytes = 1024;                      // 256 columns of B
 constexpr int kUeSfSlotBytes = kUeSfaBytes + kUeSfbBytes;
 constexpr int kUeSfColsPerSlot = 12;                   // TMEM: 4 (A) + 8 (B)
 constexpr int kUeSfGroup = 4;                          // K blocks per scale-factor slot (one byte each)
-constexpr int kUeRawSlots = 8;                         // FP32 scales as loaded
-constexpr int kUeRawFloats = kBM + 4;                  // sa of 128 rows + 2 sb (16-byte padded)
 constexpr int kUeAccCols = kUeBN;                      // one FP32 accumulator
 constexpr int kUeTmemCols = 512;
 constexpr int kUeEpiWarps = 8;
@@ -62,7 +63,7 @@ static_assert(kUeAccCols + kUeSfSlots * kUeSfColsPerSlot <= kUeTmemCols, "TMEM b
 
 constexpr int ue8m0_smem_bytes() {
     return 1024 + kUeStages * (kTileABytes + kUeTileBBytes) + kUeEpiWarps * kStageOutBytes +
-           kUeSfSlots * kUeSfSlotBytes + kUeRawSlots * kUeRawFloats * 4 + 512;
+           kUeSfSlots * kUeSfSlotBytes + 512;
 }
 
 // UE8M0 code of a positive normal power of two; anything else raises the
@@ -74,6 +75,16 @@ __device__ __forceinline__ uint32_t ue8m0_code(float v) {
     return e;
 }
 
+// Copies ring slot `slot` of the scale factors (A's 128 rows, B's two
+// 128-column blocks) from shared memory to its TMEM columns.  One thread.
+__device__ __forceinline__ void copy_sf_slot(const uint8_t* sSF, uint32_t tmem_base, int slot) {
+    const uint32_t sf_col = tmem_base + static_cast<uint32_t>(kUeAccCols + slot * kUeSfColsPerSlot);
+    const uint32_t sf_smem = smem_u32(sSF + slot * kUeSfSlotBytes);
+    tmem_cp_sf_block(sf_col, sdesc_sf_block(sf_smem));
+    tmem_cp_sf_block(sf_col + 4, sdesc_sf_block(sf_smem + kUeSfaBytes));
+    tmem_cp_sf_block(sf_col + 8, sdesc_sf_block(sf_smem + kUeSfaBytes + 512));
+}
+
 __global__ void __launch_bounds__(kUeThreads, 1)
 fp8_gemm_ue8m0_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtensorMap tmA,
                       const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmD) {
@@ -83,14 +94,11 @@ fp8_gemm_ue8m0_kernel(const __grid_constant__ Params p, const __grid_constant__ 
     uint8_t* sB = sA + kUeStages * kTileABytes;
     uint8_t* sOut = sB + kUeStages * kUeTileBBytes;
     uint8_t* sSF = sOut + kUeEpiWarps * kStageOutBytes;  // 512-byte aligned
-    float* sRaw = reinterpret_cast<float*>(sSF + kUeSfSlots * kUeSfSlotBytes);
-    uint64_t* full = reinterpret_cast<uint64_t*>(sRaw + kUeRawSlots * kUeRawFloats);
+    uint64_t* full = reinterpret_cast<uint64_t*>(sSF + kUeSfSlots * kUeSfSlotBytes);
     uint64_t* empty = full + kUeStages;
     uint64_t* sf_full = empty + kUeStages;
     uint64_t* sf_empty = sf_full + kUeSfSlots;
-    uint64_t* raw_full = sf_empty + kUeSfSlots;
-    uint64_t* raw_empty = raw_full + kUeRawSlots;
-    uint64_t* acc_full = raw_empty + kUeRawSlots;
+    uint64_t* acc_full = sf_empty + kUeSfSlots;
     uint64_t* acc_empty = acc_full + 1;
     uint64_t* done = acc_empty + 1;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
@@ -107,10 +115,6 @@ fp8_gemm_ue8m0_kernel(const __grid_constant__ Params p, const __grid_constant__ 
         for (int s = 0; s < kUeSfSlots; ++s) {
             mbar_init(sf_full + s, 1);
             mbar_init(sf_empty + s, 1);
-        }
-        for (int s = 0; s < kUeRawSlots; ++s) {
-            mbar_init(raw_full + s, 32);
-            mbar_init(raw_empty + s, 1);
         }
         mbar_init(acc_full, 1);
         mbar_init(acc_empty, kUeEpiWarps);
@@ -145,10 +149,11 @@ fp8_gemm_ue8m0_kernel(const __grid_constant__ Params p, const __grid_constant__ 
             int stage = 0, fills = 0;
             uint32_t phase = 0;
             bool ok = true;
-            for (int t = blockIdx.x; ok && t < tiles; t += gridDim.x) {
+            Work w;
+            for (int it = 0; ok && next_work(p, tiles, it, w); ++it) {
                 int mb, nb;
-                raster_tile(t, p.m_blocks, p.n_blocks, p.raster, mb, nb);
-                for (int kb = 0; kb < nkb; ++kb) {
+                raster_tile(w.t, p.m_blocks, p.n_blocks, p.raster, mb, nb);
+                for (int kb = w.kb0; kb < w.kb1; ++kb) {
                     if (!mbar_wait(empty + stage, phase ^ 1u, abort_flag)) { ok = false; break; }
                     if (lane == 0) {
                         mbar_arrive_expect_tx(full + stage, kTileABytes + kUeTileBBytes);
@@ -168,26 +173,22 @@ fp8_gemm_ue8m0_kernel(const __grid_constant__ Params p, const __grid_constant__ 
             __syncwarp();
         } else if (warp == 1) {
             // ----------------------------------------------------------- MMA ----
-            int stage = 0, slot = 0, tiles_done = 0;
+            int stage = 0, slot = 0, items = 0;
             uint32_t phase = 0, sphase = 0;
             bool ok = true;
-            for (int t = blockIdx.x; ok && t < tiles; t += gridDim.x, ++tiles_done) {
-                // The accumulator is free once the epilogue has read the previous tile.
-                if (!mbar_wait(acc_empty, (tiles_done & 1) ^ 1u, abort_flag)) { ok = false; break; }
+            Work w;
+            for (int it = 0; ok && next_work(p, tiles, it, w); ++it, ++items) {
+                // The accumulator is free once the epilogue has read the previous work item.
+                if (!mbar_wait(acc_empty, (items & 1) ^ 1u, abort_flag)) { ok = false; break; }
                 tc_fence_after();
-                for (int kb = 0; kb < nkb; ++kb) {
-                    const int j = kb % kUeSfGroup;  // byte of the scale words this K block uses
+                for (int kb = w.kb0; kb < w.kb1; ++kb) {
+                    const int j = (kb - w.kb0) % kUeSfGroup;  // byte of the scale words this K block uses
                     const uint32_t sf_col = static_cast<uint32_t>(kUeAccCols + slot * kUeSfColsPerSlot);
                     if (j == 0) {
                         // Scale factors of this group of K blocks: shared memory -> TMEM.
                         if (!mbar_wait(sf_full + slot, sphase, abort_flag)) { ok = false; break; }
                         tc_fence_after();
-                        if (lane == 0) {
-                            const uint32_t sf_smem = smem_u32(sSF + slot * kUeSfSlotBytes);
-                            tmem_cp_sf_block(tmem_base + sf_col, sdesc_sf_block(sf_smem));
-                            tmem_cp_sf_block(tmem_base + sf_col + 4, sdesc_sf_block(sf_smem + kUeSfaBytes));
-                            tmem_cp_sf_block(tmem_base + sf_col + 8, sdesc_sf_block(sf_smem + kUeSfaBytes + 512));
-                        }
+                        if (lane == 0) copy_sf_slot(sSF, tmem_base, slot);
                         __syncwarp();
                     }
                     if (!mbar_wait(full + stage, phase, abort_flag)) { ok = false; break; }
@@ -200,14 +201,14 @@ fp8_gemm_ue8m0_kernel(const __grid_constant__ Params p, const __grid_constant__ 
                         for (int k = 0; k < kBK / 32; ++k)
                             umma_f8_block_scaled(tmem_base, sdesc_kmajor_sw128(a_addr + k * 32),
                                                  sdesc_kmajor_sw128(b_addr + k * 32), idesc, tmem_base + sf_col,
-                                                 tmem_base + sf_col + 4, (kb > 0 || k > 0) ? 1u : 0u);
+                                                 tmem_base + sf_col + 4, (kb > w.kb0 || k > 0) ? 1u : 0u);
                         umma_commit(empty + stage);
-                        if (j == kUeSfGroup - 1 || kb == nkb - 1) umma_commit(sf_empty + slot);
-                        if (kb == nkb - 1) umma_commit(acc_full);
+                        if (j == kUeSfGroup - 1 || kb == w.kb1 - 1) umma_commit(sf_empty + slot);
+                        if (kb == w.kb1 - 1) umma_commit(acc_full);
                     }
                     __syncwarp();
                     if (++stage == kUeStages) { stage = 0; phase ^= 1u; }
-                    if (j == kUeSfGroup - 1 || kb == nkb - 1) {
+                    if (j == kUeSfGroup - 1 || kb == w.kb1 - 1) {
                         if (++slot == kUeSfSlots) { slot = 0; sphase ^= 1u; }
                     }
                 }
@@ -217,78 +218,58 @@ fp8_gemm_ue8m0_kernel(const __grid_constant__ Params p, const __grid_constant__ 
                 mbar_wait_drain(done, 0);
             }
             __syncwarp();
-        } else if (warp == 2) {
-            // ---------------------------------------------- scale loader ----
-            // Per K block: lane l copies sa rows m0+4l..m0+4l+3 (16 bytes) and
-            // lanes 0-1 the two sb values of the tile, asynchronously; the
-            // copies complete the slot's barrier when they land, so this warp
-            // only ever waits for a free slot.  Rows past M and blocks past
-            // N are zero-filled (and never used).
-            int slot = 0;
-            uint32_t rphase = 0;
-            bool ok = true;
-            for (int t = blockIdx.x; ok && t < tiles; t += gridDim.x) {
-                int mb, nb;
-                raster_tile(t, p.m_blocks, p.n_blocks, p.raster, mb, nb);
-                const int r4 = mb * kBM + lane * 4;
-                const int left = p.M - r4;
-                const uint32_t sa_bytes = left >= 4 ? 16u : (left > 0 ? static_cast<uint32_t>(left) * 4u : 0u);
-                const int nbl = nb * (kUeBN / 128) + (lane & 1);
-                const bool nb_ok = nbl < p.nbn;
-                for (int kb = 0; kb < nkb; ++kb) {
-                    if (!mbar_wait(raw_empty + slot, rphase ^ 1u, abort_flag)) { ok = false; break; }
-                    const uint32_t dst = smem_u32(sRaw + slot * kUeRawFloats);
-                    const float* src = sa_bytes ? p.sa + static_cast<int64_t>(kb) * p.sa_stride + r4 : p.sa;
-                    cp_async_16(dst + lane * 16, src, sa_bytes);
-                    if (lane < 2)
-                        cp_async_4(dst + (kBM + lane) * 4, nb_ok ? p.sb + static_cast<int64_t>(nbl) * nkb + kb : p.sb,
-                                   nb_ok ? 4u : 0u);
-                    cp_async_arrive(raw_full + slot);
-                    if (++slot == kUeRawSlots) { slot = 0; rphase ^= 1u; }
-                }
-            }
-            asm volatile("cp.async.wait_all;" ::: "memory");
         } else {
-            // -------------------------------------------- scale converter ----
-            // FP32 scales -> UE8M0 codes in the scale-factor layout: lane l
-            // writes line l of each block (A rows l + 32c, c < 4; B's two
-            // 128-column blocks).  Rows past M / blocks past N get code 127
-            // (a scale of 1) and only meet zero-filled operands.
-            int rslot = 0, sslot = 0;
-            uint32_t rphase = 0, sphase = 0;
+            // ------------------------------------------ scale converters ----
+            // The CTA's g-th group of kUeSfGroup K blocks, counted over its
+            // work items in order, goes to warp 2 + g % 2 and to ring slot
+            // g % kUeSfSlots.  For its group a warp reads the FP32 scales from
+            // global memory -- lane l the sa of rows m0 + l + 32c (c < 4) and
+            // the sb of the tile's two 128-column blocks, for each K block of
+            // the group -- and writes their UE8M0 codes in the scale-factor
+            // layout, lane l line l of each block.  Byte j of a word is the
+            // code of K block kb0 + j.  Entries past the data (rows past M,
+            // blocks past N, K blocks past the end) read as 1.0, code 127, and
+            // only meet zero-filled operands or unused bytes.  The loads are
+            // issued before the wait for the slot, which hides their latency.
+            const int cw = warp - 2;
+            int g = 0;
             bool ok = true;
-            for (int t = blockIdx.x; ok && t < tiles; t += gridDim.x) {
+            Work w;
+            for (int it = 0; ok && next_work(p, tiles, it, w); ++it) {
                 int mb, nb;
-                raster_tile(t, p.m_blocks, p.n_blocks, p.raster, mb, nb);
+                raster_tile(w.t, p.m_blocks, p.n_blocks, p.raster, mb, nb);
                 const int m0 = mb * kBM;
                 const int nb0 = nb * (kUeBN / 128);
-                for (int kb0 = 0; kb0 < nkb; kb0 += kUeSfGroup) {
-                    // One slot holds kUeSfGroup K blocks: byte j of every word
-                    // is the code of K block kb0 + j (127 where the tile has
-                    // fewer K blocks left).
-                    if (!mbar_wait(sf_empty + sslot, sphase ^ 1u, abort_flag)) { ok = false; break; }
-                    uint32_t a[4] = {0u, 0u, 0u, 0u}, b0 = 0u, b1 = 0u;
-#pragma unroll 1
-                    for (int j = 0; j < kUeSfGroup; ++j) {
-                        uint32_t ca[4] = {127u, 127u, 127u, 127u}, cb0 = 127u, cb1 = 127u;
-                        if (kb0 + j < nkb) {
-                            if (!mbar_wait(raw_full + rslot, rphase, abort_flag)) { ok = false; break; }
-                            const float* raw = sRaw + rslot * kUeRawFloats;
+                for (int kb0 = w.kb0; kb0 < w.kb1; kb0 += kUeSfGroup, ++g) {
+                    if ((g & 1) != cw) continue;
+                    float fa[kUeSfGroup][4], fb[kUeSfGroup][2];
 #pragma unroll
-                            for (int c = 0; c < 4; ++c)
-                                if (m0 + lane + 32 * c < p.M) ca[c] = ue8m0_code(raw[lane + 32 * c]);
-                            if (nb0 < p.nbn) cb0 = ue8m0_code(raw[kBM]);
-                            if (nb0 + 1 < p.nbn) cb1 = ue8m0_code(raw[kBM + 1]);
-                            __syncwarp();
-                            if (lane == 0) mbar_arrive(raw_empty + rslot);
-                            if (++rslot == kUeRawSlots) { rslot = 0; rphase ^= 1u; }
+                    for (int j = 0; j < kUeSfGroup; ++j) {
+                        const bool kb_ok = kb0 + j < w.kb1;
+#pragma unroll
+                        for (int c = 0; c < 4; ++c) {
+                            const int row = m0 + lane + 32 * c;
+                            fa[j][c] = (kb_ok && row < p.M)
+                                           ? __ldg(p.sa + static_cast<int64_t>(kb0 + j) * p.sa_stride + row)
+                                           : 1.0f;
                         }
 #pragma unroll
-                        for (int c = 0; c < 4; ++c) a[c] |= ca[c] << (8 * j);
-                        b0 |= cb0 << (8 * j);
-                        b1 |= cb1 << (8 * j);
+                        for (int h = 0; h < 2; ++h)
+                            fb[j][h] = (kb_ok && nb0 + h < p.nbn)
+                                           ? __ldg(p.sb + static_cast<int64_t>(nb0 + h) * nkb + kb0 + j)
+                                           : 1.0f;
                     }
-                    if (!ok) break;
+                    const int sslot = g % kUeSfSlots;
+                    const uint32_t sphase = static_cast<uint32_t>(g / kUeSfSlots) & 1u;
+                    if (!mbar_wait(sf_empty + sslot, sphase ^ 1u, abort_flag)) { ok = false; break; }
+                    uint32_t a[4] = {0u, 0u, 0u, 0u}, b0 = 0u, b1 = 0u;
+#pragma unroll
+                    for (int j = 0; j < kUeSfGroup; ++j) {
+#pragma unroll
+                        for (int c = 0; c < 4; ++c) a[c] |= ue8m0_code(fa[j][c]) << (8 * j);
+                        b0 |= ue8m0_code(fb[j][0]) << (8 * j);
+                        b1 |= ue8m0_code(fb[j][1]) << (8 * j);
+                    }
                     const uint32_t base = smem_u32(sSF + sslot * kUeSfSlotBytes);
                     st_shared_v4(base + lane * 16, a[0], a[1], a[2], a[3]);
                     st_shared_v4(base + kUeSfaBytes + lane * 16, b0, b0, b0, b0);
@@ -296,7 +277,6 @@ fp8_gemm_ue8m0_kernel(const __grid_constant__ Params p, const __grid_constant__ 
                     fence_proxy_async_smem();  // the copy to TMEM reads through the async proxy
                     __syncwarp();
                     if (lane == 0) mbar_arrive(sf_full + sslot);
-                    if (++sslot == kUeSfSlots) { sslot = 0; sphase ^= 1u; }
                 }
             }
         }
@@ -307,12 +287,13 @@ fp8_gemm_ue8m0_kernel(const __grid_constant__ Params p, const __grid_constant__ 
         const int half = ew >> 2;  // 128-column half of the tile
         const int quarter = warp & 3;
         const uint32_t t_lane = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16);
-        int tiles_done = 0;
+        int items = 0;
         bool ok = true;
-        for (int t = blockIdx.x; ok && t < tiles; t += gridDim.x, ++tiles_done) {
+        Work w;
+        for (int it = 0; ok && next_work(p, tiles, it, w); ++it, ++items) {
             int mb, nb;
-            raster_tile(t, p.m_blocks, p.n_blocks, p.raster, mb, nb);
-            if (!mbar_wait(acc_full, tiles_done & 1, abort_flag)) { ok = false; break; }
+            raster_tile(w.t, p.m_blocks, p.n_blocks, p.raster, mb, nb);
+            if (!mbar_wait(acc_full, items & 1, abort_flag)) { ok = false; break; }
             tc_fence_after();
             uint32_t v[4][32];
 #pragma unroll
@@ -322,7 +303,51 @@ fp8_gemm_ue8m0_kernel(const __grid_constant__ Params p, const __grid_constant__ 
             for (int c = 0; c < 4; ++c) reg_fence(v[c]);
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(acc_empty);  // the MMA may start the next tile
+            if (lane == 0) mbar_arrive(acc_empty);  // the MMA may start the next work item
+            if (w.slice >= 0) {
+                // K slice of a split tile.  Partial (r, s) for slices s >= 1
+                // lives at ws + (r*(S-1) + s-1) * 128*256 floats in the layout
+                // [epilogue warp][float4 j][lane] (float4 j = columns 4j..4j+3
+                // of the warp's 128).  Slice s >= 1 writes its partial and
+                // raises its flag; slice 0 waits for every flag, adds the
+                // partials in slice order (so the result does not depend on
+                // timing), clears the flags and stores D.
+                const int S = p.tail_split;
+                const int rt = w.t - p.full_tiles;
+                const bool leader = (warp == kFirstEpiWarp && lane == 0);
+                if (w.slice > 0) {
+                    float4* dst = reinterpret_cast<float4*>(p.ws + static_cast<int64_t>(rt * (S - 1) + w.slice - 1) * kBM * kUeBN);
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        const uint32_t* q = &v[j >> 3][(j & 7) * 4];
+                        __stcg(dst + (ew * 32 + j) * 32 + lane, make_float4(__uint_as_float(q[0]), __uint_as_float(q[1]),
+                                                                            __uint_as_float(q[2]), __uint_as_float(q[3])));
+                    }
+                    __threadfence();
+                    named_barrier_sync(1, 32 * kUeEpiWarps);
+                    if (leader) st_release_gpu(p.ws_flags + rt * (S - 1) + w.slice - 1, 1u);
+                    continue;  // slice 0 stores the tile
+                }
+                bool got = true;
+                if (leader) {
+                    for (int s2 = 1; s2 < S && got; ++s2) got = wait_flag_gpu(p.ws_flags + rt * (S - 1) + s2 - 1);
+                    for (int s2 = 1; s2 < S; ++s2) p.ws_flags[rt * (S - 1) + s2 - 1] = 0u;
+                    if (!got) atomicOr(&g_dg_error, 1u);
+                }
+                named_barrier_sync(1, 32 * kUeEpiWarps);
+                for (int s2 = 1; s2 < S; ++s2) {
+                    const float4* src = reinterpret_cast<const float4*>(p.ws + static_cast<int64_t>(rt * (S - 1) + s2 - 1) * kBM * kUeBN);
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        const float4 a = __ldcg(src + (ew * 32 + j) * 32 + lane);
+                        uint32_t* q = &v[j >> 3][(j & 7) * 4];
+                        q[0] = __float_as_uint(__uint_as_float(q[0]) + a.x);
+                        q[1] = __float_as_uint(__uint_as_float(q[1]) + a.y);
+                        q[2] = __float_as_uint(__uint_as_float(q[2]) + a.z);
+                        q[3] = __float_as_uint(__uint_as_float(q[3]) + a.w);
+                    }
+                }
+            }
             // bf16, staged 32 rows x 32 columns at a time with the 64-byte
             // swizzle of the output map, one TMA store per piece.
             const uint32_t stg = smem_u32(sOut + ew * kStageOutBytes);

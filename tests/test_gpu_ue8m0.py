@@ -87,9 +87,30 @@ def test_scales_that_are_not_powers_of_two_are_flagged(dgm):
     assert dgm.dg_get_device_error() == 0
 
 
-def test_routing_keeps_the_result(monkeypatch, dgm):
-    # Unforced, a long-K shape takes the promotion kernel: same sum.
-    monkeypatch.setenv("DG_FORCE_BLOCK_SCALED", "0")
-    c = wl.dense_case(256, 512, 4096, seed=9, stress=True)
+@pytest.mark.parametrize("sms", [148, 7, 4])
+def test_ue8m0_k_split(dgm, sms):
+    # 300 x 520 x 6144: 3 x 3 tiles of 128 x 256 and 48 K blocks.  On 148 SMs
+    # all nine tiles are split into 3 K slices (27 CTAs); on 7 SMs the two
+    # tiles after one full wave are, on 4 SMs the one tile after two waves.
+    c = wl.dense_case(300, 520, 6144, seed=11, stress=True)
+    dgm.dg_set_num_sms(sms)
+    try:
+        got = _run(dgm, c)
+        again = _run(dgm, c)
+    finally:
+        dgm.dg_set_num_sms(0)
+    assert dgm.dg_get_device_error() == 0
+    assert dgm.dg_get_workspace_count() >= 1, "the split ran without its workspace"
+    assert np.array_equal(got, again), "split result differs between runs"
+    _check(got, c, None, f"ue8m0 split on {sms} SMs")
+
+
+@pytest.mark.parametrize("M", [128, 256, 384])
+def test_routing_keeps_the_result(monkeypatch, dgm, M):
+    # Unforced, up to 256 rows take the promotion path and more the
+    # block-scaled kernel: the same sum either way.
+    monkeypatch.delenv("DG_FORCE_BLOCK_SCALED", raising=False)
+    c = wl.dense_case(M, 512, 4096, seed=9, stress=True)
     got = _run(dgm, c)
-    _check(got, c, None, "routed ue8m0 call")
+    assert dgm.dg_get_device_error() == 0
+    _check(got, c, None, f"routed ue8m0 call, M={M}")
