@@ -311,11 +311,15 @@ class Ue8m0Problem(Problem):
         if self.path == "promote":
             self.dg.dg_fp8_gemm_nt(D, c.A, c.sa, c.sa_stride, c.B, c.sb)
         else:
-            os.environ["DG_FORCE_BLOCK_SCALED"] = "1" if self.path == "block_scaled" else "0"
+            prev = os.environ.pop("DG_FORCE_BLOCK_SCALED", None)
+            if self.path == "block_scaled":
+                os.environ["DG_FORCE_BLOCK_SCALED"] = "1"
             try:
                 self.dg.dg_fp8_gemm_nt_ue8m0(D, c.A, c.sa, c.sa_stride, c.B, c.sb)
             finally:
                 os.environ.pop("DG_FORCE_BLOCK_SCALED", None)
+                if prev is not None:
+                    os.environ["DG_FORCE_BLOCK_SCALED"] = prev
 
 
 # The block-scaled comparison shapes; the last two are the stress workload
