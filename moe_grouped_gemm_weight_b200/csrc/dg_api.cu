@@ -975,6 +975,16 @@ dg_status dg_fp8_gemm_nt_ue8m0(uint16_t* D, const uint8_t* A, const float* sa, i
     if (dev >= 0 && dev < kMaxDevices && !attr_set[dev].load()) {
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
             return fail(DG_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(cudaGetLastError()));
+        // The kernel's setmaxnreg split draws on the registers the CTA is
+        // launched with (its threads x the compiled register count); a build
+        // whose count cannot cover the split would wait forever in
+        // setmaxnreg, so it is refused here, before any launch.
+        cudaFuncAttributes fa{};
+        if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess)
+            return fail(DG_ERR_CUDA, "cudaFuncGetAttributes: %s", cudaGetErrorString(cudaGetLastError()));
+        if (fa.numRegs < dg::kUeLaunchRegsNeeded)
+            return fail(DG_ERR_UNSUPPORTED, "block-scaled kernel compiled with %d registers per thread, its register "
+                        "split needs %d", fa.numRegs, dg::kUeLaunchRegsNeeded);
         attr_set[dev].store(1);
     }
     cudaLaunchConfig_t cfg = {};

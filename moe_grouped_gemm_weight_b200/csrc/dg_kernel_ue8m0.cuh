@@ -18,21 +18,26 @@
 // (section 3.1) notes that on SM100 the scales are UE8M0.  This kernel is the
 // SM100 path for such scales; the general FP32-scale kernels stay the default.
 //
-// Tiles 128 x 256, persistent CTAs of 384 threads.  The work items are those
+// Tiles 128 x 256, persistent CTAs of 512 threads (four warpgroups, so that
+// every warpgroup executes one setmaxnreg: 56 registers for the first two,
+// 200 for the epilogue's two).  The work items are those
 // of the promotion kernel: whole tiles round-robin, and, when the planner asks
 // for it, the tiles of the last partial wave (or all tiles, when there are
 // fewer than CTAs) split into K slices whose FP32 partials slice 0 adds up.
 //   warp 0      TMA producer (A 128x128 and B 256x128 per K block, 4 stages)
-//   warp 1      TMEM owner; per four K blocks copies their scale factors from
-//               shared memory to TMEM (tcgen05.cp); per K block issues 4 MMAs
-//   warps 2-3   scale converters, taking alternate groups of four K blocks:
+//   warps 1-2   MMA issuers, taking alternate K blocks (warp 1 also owns
+//               TMEM); the K block that starts a group of four first copies
+//               the group's scale factors from shared memory to TMEM
+//               (tcgen05.cp); each K block is 4 MMAs into the one accumulator
+//   warps 4-5   scale converters, taking alternate groups of four K blocks:
 //               FP32 sa (128 rows) and sb (2 blocks) read from global memory,
 //               UE8M0 codes written in the scale-factor layout, 8-slot ring;
 //               a scale that is not a positive normal power of two sets
 //               DG_DEVERR_NOT_POW2 (its code is still its exponent field, so
 //               the result is wrong for it)
-//   warps 4-11  epilogue: TMEM -> bf16 -> TMA store (two warpgroups of 128
-//               columns)
+//   warps 8-15  epilogue: TMEM -> bf16 -> TMA store (two warpgroups of 128
+//               columns; warp w reads TMEM lanes 32 * (w % 4) onwards)
+//   warps 3, 6, 7 have no role.
 // Scale-factor layout in shared memory (one 512-byte block per 128 rows or
 // columns): the 32-bit word for row r sits at byte (r % 32) * 16 + (r / 32) * 4.
 // tcgen05.cp .32x128b.warpx4 places it in TMEM column (r / 32) of lane r % 32,
@@ -56,8 +61,20 @@ constexpr int kUeSfColsPerSlot = 12;                   // TMEM: 4 (A) + 8 (B)
 constexpr int kUeSfGroup = 4;                          // K blocks per scale-factor slot (one byte each)
 constexpr int kUeAccCols = kUeBN;                      // one FP32 accumulator
 constexpr int kUeTmemCols = 512;
+constexpr int kUeFirstEpiWarp = 8;                     // warpgroups 0-1: producer, MMA, converters
 constexpr int kUeEpiWarps = 8;
-constexpr int kUeThreads = 32 * (kFirstEpiWarp + kUeEpiWarps);
+constexpr int kUeThreads = 32 * (kUeFirstEpiWarp + kUeEpiWarps);
+static_assert(kUeFirstEpiWarp % 4 == 0 && kUeEpiWarps % 4 == 0, "setmaxnreg works on whole warpgroups");
+// setmaxnreg budgets: the first two warpgroups give registers to the
+// epilogue's two.  Their sum over all threads must stay within the registers
+// the CTA is launched with (kUeThreads x the kernel's register count); the
+// host checks the compiled count against kUeLaunchRegsNeeded before the first
+// launch.
+constexpr int kUeRegsLow = 56;
+constexpr int kUeRegsHigh = 200;
+constexpr int kUeRegsTotal = 32 * (kUeFirstEpiWarp * kUeRegsLow + kUeEpiWarps * kUeRegsHigh);
+constexpr int kUeLaunchRegsNeeded = (kUeRegsTotal + kUeThreads - 1) / kUeThreads;
+static_assert(kUeRegsTotal <= 65536, "register split exceeds the file");
 constexpr int kUeTileBBytes = kUeBN * kBK;
 static_assert(kUeAccCols + kUeSfSlots * kUeSfColsPerSlot <= kUeTmemCols, "TMEM budget");
 
@@ -100,8 +117,9 @@ fp8_gemm_ue8m0_kernel(const __grid_constant__ Params p, const __grid_constant__ 
     uint64_t* sf_empty = sf_full + kUeSfSlots;
     uint64_t* acc_full = sf_empty + kUeSfSlots;
     uint64_t* acc_empty = acc_full + 1;
-    uint64_t* done = acc_empty + 1;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+    uint64_t* done = acc_empty + 1;   // [2], one per MMA warp
+    uint64_t* hand = done + 2;        // [2]: MMA warp w has issued its latest K block
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(hand + 2);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5;
@@ -118,7 +136,10 @@ fp8_gemm_ue8m0_kernel(const __grid_constant__ Params p, const __grid_constant__ 
         }
         mbar_init(acc_full, 1);
         mbar_init(acc_empty, kUeEpiWarps);
-        mbar_init(done, 1);
+        for (int w2 = 0; w2 < 2; ++w2) {
+            mbar_init(done + w2, 1);
+            mbar_init(hand + w2, 1);
+        }
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -140,8 +161,8 @@ fp8_gemm_ue8m0_kernel(const __grid_constant__ Params p, const __grid_constant__ 
     const int tiles = p.m_blocks * p.n_blocks;
     const int nkb = p.nkb;
 
-    if (warp < kFirstEpiWarp) {
-        regs_dec<56>();
+    if (warp < kUeFirstEpiWarp) {
+        regs_dec<kUeRegsLow>();
         if (warp == 0) {
             // ------------------------------------------------------ producer ----
             const uint64_t pol_a = l2_policy_evict_last();
@@ -171,57 +192,73 @@ fp8_gemm_ue8m0_kernel(const __grid_constant__ Params p, const __grid_constant__ 
                     mbar_wait_drain(full + (i % kUeStages), static_cast<uint32_t>((i / kUeStages) & 1));
             }
             __syncwarp();
-        } else if (warp == 1) {
+        } else if (warp == 1 || warp == 2) {
             // ----------------------------------------------------------- MMA ----
-            int stage = 0, slot = 0, items = 0;
+            // Two warps issue the MMAs of alternate K blocks (the CTA's i-th K
+            // block, counted over its work items, goes to warp 1 + i % 2).  A
+            // warp waits for its operand stage (and, at a group start, copies
+            // the scale factors) while the other issues; the hand-over keeps
+            // the MMAs into the one accumulator in K order: the issuer of
+            // block i fences and arrives on hand[its warp] once its MMAs and
+            // commits are issued, and block i+1's issuer waits for that
+            // arrival and fences before its first MMA.
+            const int mw = warp - 1;
+            int stage = 0, slot = 0, items = 0, i = 0;
             uint32_t phase = 0, sphase = 0;
             bool ok = true;
             Work w;
             for (int it = 0; ok && next_work(p, tiles, it, w); ++it, ++items) {
-                // The accumulator is free once the epilogue has read the previous work item.
-                if (!mbar_wait(acc_empty, (items & 1) ^ 1u, abort_flag)) { ok = false; break; }
-                tc_fence_after();
-                for (int kb = w.kb0; kb < w.kb1; ++kb) {
+                for (int kb = w.kb0; kb < w.kb1; ++kb, ++i) {
                     const int j = (kb - w.kb0) % kUeSfGroup;  // byte of the scale words this K block uses
-                    const uint32_t sf_col = static_cast<uint32_t>(kUeAccCols + slot * kUeSfColsPerSlot);
-                    if (j == 0) {
-                        // Scale factors of this group of K blocks: shared memory -> TMEM.
-                        if (!mbar_wait(sf_full + slot, sphase, abort_flag)) { ok = false; break; }
+                    const bool group_end = j == kUeSfGroup - 1 || kb == w.kb1 - 1;
+                    if ((i & 1) == mw) {
+                        const uint32_t sf_col = static_cast<uint32_t>(kUeAccCols + slot * kUeSfColsPerSlot);
+                        if (kb == w.kb0) {
+                            // The accumulator is free once the epilogue has read the previous work item.
+                            if (!mbar_wait(acc_empty, (items & 1) ^ 1u, abort_flag)) { ok = false; break; }
+                        }
+                        if (!mbar_wait(full + stage, phase, abort_flag)) { ok = false; break; }
+                        if (j == 0 && !mbar_wait(sf_full + slot, sphase, abort_flag)) { ok = false; break; }
+                        if (i > 0) {
+                            // Block i-1 was the other warp's: its ((i + mw) / 2)-th hand-over.
+                            const uint32_t hp = static_cast<uint32_t>((i + mw) / 2 - 1) & 1u;
+                            if (!mbar_wait(hand + (1 - mw), hp, abort_flag)) { ok = false; break; }
+                        }
                         tc_fence_after();
-                        if (lane == 0) copy_sf_slot(sSF, tmem_base, slot);
-                        __syncwarp();
-                    }
-                    if (!mbar_wait(full + stage, phase, abort_flag)) { ok = false; break; }
-                    tc_fence_after();
-                    if (lane == 0) {
-                        const uint32_t a_addr = smem_u32(sA + stage * kTileABytes);
-                        const uint32_t b_addr = smem_u32(sB + stage * kUeTileBBytes);
-                        const uint32_t idesc = idesc_e4m3_ue8m0(kBM, kUeBN, j, j);
+                        if (lane == 0) {
+                            if (j == 0) copy_sf_slot(sSF, tmem_base, slot);
+                            const uint32_t a_addr = smem_u32(sA + stage * kTileABytes);
+                            const uint32_t b_addr = smem_u32(sB + stage * kUeTileBBytes);
+                            const uint32_t idesc = idesc_e4m3_ue8m0(kBM, kUeBN, j, j);
 #pragma unroll
-                        for (int k = 0; k < kBK / 32; ++k)
-                            umma_f8_block_scaled(tmem_base, sdesc_kmajor_sw128(a_addr + k * 32),
-                                                 sdesc_kmajor_sw128(b_addr + k * 32), idesc, tmem_base + sf_col,
-                                                 tmem_base + sf_col + 4, (kb > w.kb0 || k > 0) ? 1u : 0u);
-                        umma_commit(empty + stage);
-                        if (j == kUeSfGroup - 1 || kb == w.kb1 - 1) umma_commit(sf_empty + slot);
-                        if (kb == w.kb1 - 1) umma_commit(acc_full);
+                            for (int k = 0; k < kBK / 32; ++k)
+                                umma_f8_block_scaled(tmem_base, sdesc_kmajor_sw128(a_addr + k * 32),
+                                                     sdesc_kmajor_sw128(b_addr + k * 32), idesc, tmem_base + sf_col,
+                                                     tmem_base + sf_col + 4, (kb > w.kb0 || k > 0) ? 1u : 0u);
+                            umma_commit(empty + stage);
+                            if (group_end) umma_commit(sf_empty + slot);
+                            if (kb == w.kb1 - 1) umma_commit(acc_full);
+                        }
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(hand + mw);
                     }
-                    __syncwarp();
                     if (++stage == kUeStages) { stage = 0; phase ^= 1u; }
-                    if (j == kUeSfGroup - 1 || kb == w.kb1 - 1) {
+                    if (group_end) {
                         if (++slot == kUeSfSlots) { slot = 0; sphase ^= 1u; }
                     }
                 }
             }
+            // All MMAs of this warp must have finished before TMEM is released.
             if (lane == 0) {
-                umma_commit(done);
-                mbar_wait_drain(done, 0);
+                umma_commit(done + mw);
+                mbar_wait_drain(done + mw, 0);
             }
             __syncwarp();
-        } else {
+        } else if (warp == 4 || warp == 5) {
             // ------------------------------------------ scale converters ----
             // The CTA's g-th group of kUeSfGroup K blocks, counted over its
-            // work items in order, goes to warp 2 + g % 2 and to ring slot
+            // work items in order, goes to warp 4 + g % 2 and to ring slot
             // g % kUeSfSlots.  For its group a warp reads the FP32 scales from
             // global memory -- lane l the sa of rows m0 + l + 32c (c < 4) and
             // the sb of the tile's two 128-column blocks, for each K block of
@@ -229,9 +266,11 @@ fp8_gemm_ue8m0_kernel(const __grid_constant__ Params p, const __grid_constant__ 
             // layout, lane l line l of each block.  Byte j of a word is the
             // code of K block kb0 + j.  Entries past the data (rows past M,
             // blocks past N, K blocks past the end) read as 1.0, code 127, and
-            // only meet zero-filled operands or unused bytes.  The loads are
-            // issued before the wait for the slot, which hides their latency.
-            const int cw = warp - 2;
+            // only meet zero-filled operands or unused bytes.  The loads of
+            // two K blocks are in flight at a time (the warp runs in 56
+            // registers); the first pair is issued before the wait for the
+            // slot.
+            const int cw = warp - 4;
             int g = 0;
             bool ok = true;
             Work w;
@@ -242,34 +281,40 @@ fp8_gemm_ue8m0_kernel(const __grid_constant__ Params p, const __grid_constant__ 
                 const int nb0 = nb * (kUeBN / 128);
                 for (int kb0 = w.kb0; kb0 < w.kb1; kb0 += kUeSfGroup, ++g) {
                     if ((g & 1) != cw) continue;
-                    float fa[kUeSfGroup][4], fb[kUeSfGroup][2];
-#pragma unroll
-                    for (int j = 0; j < kUeSfGroup; ++j) {
-                        const bool kb_ok = kb0 + j < w.kb1;
-#pragma unroll
-                        for (int c = 0; c < 4; ++c) {
-                            const int row = m0 + lane + 32 * c;
-                            fa[j][c] = (kb_ok && row < p.M)
-                                           ? __ldg(p.sa + static_cast<int64_t>(kb0 + j) * p.sa_stride + row)
-                                           : 1.0f;
-                        }
-#pragma unroll
-                        for (int h = 0; h < 2; ++h)
-                            fb[j][h] = (kb_ok && nb0 + h < p.nbn)
-                                           ? __ldg(p.sb + static_cast<int64_t>(nb0 + h) * nkb + kb0 + j)
-                                           : 1.0f;
-                    }
                     const int sslot = g % kUeSfSlots;
                     const uint32_t sphase = static_cast<uint32_t>(g / kUeSfSlots) & 1u;
-                    if (!mbar_wait(sf_empty + sslot, sphase ^ 1u, abort_flag)) { ok = false; break; }
                     uint32_t a[4] = {0u, 0u, 0u, 0u}, b0 = 0u, b1 = 0u;
 #pragma unroll
-                    for (int j = 0; j < kUeSfGroup; ++j) {
+                    for (int jp = 0; jp < kUeSfGroup; jp += 2) {
+                        float fa[2][4], fb[2][2];
 #pragma unroll
-                        for (int c = 0; c < 4; ++c) a[c] |= ue8m0_code(fa[j][c]) << (8 * j);
-                        b0 |= ue8m0_code(fb[j][0]) << (8 * j);
-                        b1 |= ue8m0_code(fb[j][1]) << (8 * j);
+                        for (int jj = 0; jj < 2; ++jj) {
+                            const int kb = kb0 + jp + jj;
+                            const bool kb_ok = kb < w.kb1;
+#pragma unroll
+                            for (int c = 0; c < 4; ++c) {
+                                const int row = m0 + lane + 32 * c;
+                                fa[jj][c] = (kb_ok && row < p.M)
+                                                ? __ldg(p.sa + static_cast<int64_t>(kb) * p.sa_stride + row)
+                                                : 1.0f;
+                            }
+#pragma unroll
+                            for (int h = 0; h < 2; ++h)
+                                fb[jj][h] = (kb_ok && nb0 + h < p.nbn)
+                                                ? __ldg(p.sb + static_cast<int64_t>(nb0 + h) * nkb + kb)
+                                                : 1.0f;
+                        }
+                        if (jp == 0 && !mbar_wait(sf_empty + sslot, sphase ^ 1u, abort_flag)) { ok = false; break; }
+#pragma unroll
+                        for (int jj = 0; jj < 2; ++jj) {
+                            const int sh = 8 * (jp + jj);
+#pragma unroll
+                            for (int c = 0; c < 4; ++c) a[c] |= ue8m0_code(fa[jj][c]) << sh;
+                            b0 |= ue8m0_code(fb[jj][0]) << sh;
+                            b1 |= ue8m0_code(fb[jj][1]) << sh;
+                        }
                     }
+                    if (!ok) break;
                     const uint32_t base = smem_u32(sSF + sslot * kUeSfSlotBytes);
                     st_shared_v4(base + lane * 16, a[0], a[1], a[2], a[3]);
                     st_shared_v4(base + kUeSfaBytes + lane * 16, b0, b0, b0, b0);
@@ -282,8 +327,8 @@ fp8_gemm_ue8m0_kernel(const __grid_constant__ Params p, const __grid_constant__ 
         }
     } else {
         // ------------------------------------------------------- epilogue ----
-        regs_inc<224>();
-        const int ew = warp - kFirstEpiWarp;
+        regs_inc<kUeRegsHigh>();
+        const int ew = warp - kUeFirstEpiWarp;
         const int half = ew >> 2;  // 128-column half of the tile
         const int quarter = warp & 3;
         const uint32_t t_lane = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16);
@@ -314,7 +359,7 @@ fp8_gemm_ue8m0_kernel(const __grid_constant__ Params p, const __grid_constant__ 
                 // timing), clears the flags and stores D.
                 const int S = p.tail_split;
                 const int rt = w.t - p.full_tiles;
-                const bool leader = (warp == kFirstEpiWarp && lane == 0);
+                const bool leader = (warp == kUeFirstEpiWarp && lane == 0);
                 if (w.slice > 0) {
                     float4* dst = reinterpret_cast<float4*>(p.ws + static_cast<int64_t>(rt * (S - 1) + w.slice - 1) * kBM * kUeBN);
 #pragma unroll

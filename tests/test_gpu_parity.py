@@ -225,6 +225,22 @@ def test_masked_full_size_sampled(dgm, cfg):
     assert_close(flat_g[rows], flat_r[rows], mag.reshape(-1, c.N)[rows], "masked full size")
 
 
+@pytest.mark.parametrize("hint", [1, 40, 100, 200, 1000])
+def test_masked_expected_m_hint_never_changes_the_result(dgm, hint):
+    # expected_m only steers the planner's tile shape; D must match the
+    # unhinted call bit for bit (no K split is planned at these sizes, so
+    # every element is summed in the same order), and the oracle.
+    c = wl.masked_case(3, 200, 264, 512, masked_m=[0, 200, 65], seed=21)
+    base = run_masked(dgm, c, 0)
+    got = run_masked(dgm, c, hint)
+    assert dgm.dg_get_device_error() == 0
+    assert np.array_equal(got, base), f"expected_m={hint} changed D"
+    ref, mag = oracle_masked(c)
+    check_masked_untouched(got, [0, 200, 65])
+    for g, mm in enumerate([0, 200, 65]):
+        assert_close(got[g, :mm], ref[g, :mm], mag[g, :mm], f"masked hint {hint}, group {g}")
+
+
 def test_masked_count_beyond_mmax_is_clamped_and_flagged(dgm):
     c = wl.masked_case(2, 64, 64, 128, masked_m=[3, 64], seed=11)
     c.masked_m[1] = 1000
