@@ -105,6 +105,22 @@ def test_ue8m0_k_split(dgm, sms):
     _check(got, c, None, f"ue8m0 split on {sms} SMs")
 
 
+@pytest.mark.parametrize("sms", [4, 3])
+def test_ue8m0_odd_k_blocks_over_many_work_items(dgm, sms):
+    # 513 x 1032 x 640: 5 x 5 tiles of 5 K blocks each, too short to split.
+    # On 4 (3) SMs each CTA walks 6-7 (8-9) work items, so the two MMA warps'
+    # turn -- alternate K blocks, counted over the CTA's work items -- falls
+    # on the other warp at every new tile.
+    c = wl.dense_case(513, 1032, 640, seed=17, stress=True)
+    dgm.dg_set_num_sms(sms)
+    try:
+        got = _run(dgm, c)
+    finally:
+        dgm.dg_set_num_sms(0)
+    assert dgm.dg_get_device_error() == 0
+    _check(got, c, None, f"ue8m0 odd K blocks on {sms} SMs")
+
+
 @pytest.mark.parametrize("M", [128, 256, 384])
 def test_routing_keeps_the_result(monkeypatch, dgm, M):
     # Unforced, up to 256 rows take the promotion path and more the
