@@ -105,6 +105,19 @@ def test_ue8m0_k_split(dgm, sms):
     _check(got, c, None, f"ue8m0 split on {sms} SMs")
 
 
+def test_ue8m0_uneven_k_split(dgm):
+    # 300 x 520 x 6400: 9 tiles of 50 K blocks, split 3 ways on 148 SMs into
+    # slices of 16, 17 and 17 K blocks: the second and third slices start at
+    # K blocks 16 and 33, so their groups of four scale bytes start off the
+    # multiples of four.
+    c = wl.dense_case(300, 520, 6400, seed=23, stress=True)
+    got = _run(dgm, c)
+    again = _run(dgm, c)
+    assert dgm.dg_get_device_error() == 0
+    assert np.array_equal(got, again), "split result differs between runs"
+    _check(got, c, None, "ue8m0 uneven split")
+
+
 @pytest.mark.parametrize("sms", [4, 3])
 def test_ue8m0_odd_k_blocks_over_many_work_items(dgm, sms):
     # 513 x 1032 x 640: 5 x 5 tiles of 5 K blocks each, too short to split.
