@@ -36,6 +36,13 @@
 
 namespace dg {
 
+// Cluster-barrier arrive without release semantics: for a barrier that only
+// keeps the CTAs of a cluster alive until their peers are done, where nothing
+// written before the arrive is read after the wait because of it.
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+    asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+}
+
 constexpr int kSmallThreads = 384;
 constexpr int kSmallFirstEpiWarp = 4;
 constexpr int kSmallEpiWarps = 8;
@@ -497,8 +504,12 @@ fp8_gemm_swapab_kernel(const __grid_constant__ Params p, const __grid_constant__
                 }
                 // Everything this CTA receives has landed: arrive now, so the
                 // barrier that keeps each CTA alive until every copy out of it
-                // has completed overlaps the sums below.
-                cluster_arrive();
+                // has completed overlaps the sums below.  The arrive needs no
+                // release: a peer arrives only once its own receive barrier has
+                // counted our copies in, and what this CTA reads after the
+                // final wait is only its own shared memory.  (A release arrive
+                // cost ~860 cycles here, on the critical path.)
+                cluster_arrive_relaxed();
                 const float* rcv = reinterpret_cast<const float*>(aux);
                 const int rows_mine = my_j1 - my_j0;
                 for (int e = ptid; e < rows_mine * 32; e += kSmallEpiThreads) {
