@@ -512,29 +512,38 @@ fp8_gemm_swapab_kernel(const __grid_constant__ Params p, const __grid_constant__
                 cluster_arrive_relaxed();
                 const float* rcv = reinterpret_cast<const float*>(aux);
                 const int rows_mine = my_j1 - my_j0;
-                for (int e = ptid; e < rows_mine * 32; e += kSmallEpiThreads) {
-                    const int jj = e >> 5, c4 = (e & 31) * 4;
-                    float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
+                // One 8-column chunk per thread and step: a single pass for
+                // the rows a CTA owns at TN <= 64, and one 16-byte store
+                // (N % 8 == 0, so a chunk is wholly inside D or wholly past N).
+                for (int e = ptid; e < rows_mine * 16; e += kSmallEpiThreads) {
+                    const int jj = e >> 4, c8 = (e & 15) * 8;
+                    float4 sa4 = make_float4(0.f, 0.f, 0.f, 0.f), sb4 = sa4;
 #pragma unroll
                     for (int r = 0; r < C::kMaxSplit; ++r)
                         if (r < S) {
-                            const float* src = r == rank ? red + (my_j0 + jj) * 128 + c4
-                                                         : rcv + ((r < rank ? r : r - 1) * rows_mine + jj) * 128 + c4;
-                            const float4 v4 = *reinterpret_cast<const float4*>(src);
+                            const float* src = r == rank ? red + (my_j0 + jj) * 128 + c8
+                                                         : rcv + ((r < rank ? r : r - 1) * rows_mine + jj) * 128 + c8;
+                            const float4 a4 = *reinterpret_cast<const float4*>(src);
+                            const float4 b4 = *reinterpret_cast<const float4*>(src + 4);
                             if (r == 0) {
-                                sum = v4;
+                                sa4 = a4; sb4 = b4;
                             } else {
-                                sum.x += v4.x; sum.y += v4.y; sum.z += v4.z; sum.w += v4.w;
+                                sa4.x += a4.x; sa4.y += a4.y; sa4.z += a4.z; sa4.w += a4.w;
+                                sb4.x += b4.x; sb4.y += b4.y; sb4.z += b4.z; sb4.w += b4.w;
                             }
                         }
-                    const int row = tl.m0 + my_j0 + jj, col = tl.n0 + c4;
+                    const int row = tl.m0 + my_j0 + jj, col = tl.n0 + c8;
                     if (row < tl.rows && col < p.N) {
-                        __nv_bfloat162 h0 = __floats2bfloat162_rn(sum.x, sum.y);
-                        __nv_bfloat162 h1 = __floats2bfloat162_rn(sum.z, sum.w);
-                        uint2 pk;
+                        __nv_bfloat162 h0 = __floats2bfloat162_rn(sa4.x, sa4.y);
+                        __nv_bfloat162 h1 = __floats2bfloat162_rn(sa4.z, sa4.w);
+                        __nv_bfloat162 h2 = __floats2bfloat162_rn(sb4.x, sb4.y);
+                        __nv_bfloat162 h3 = __floats2bfloat162_rn(sb4.z, sb4.w);
+                        uint4 pk;
                         pk.x = *reinterpret_cast<uint32_t*>(&h0);
                         pk.y = *reinterpret_cast<uint32_t*>(&h1);
-                        *reinterpret_cast<uint2*>(p.D + (d_base + row) * p.N + col) = pk;
+                        pk.z = *reinterpret_cast<uint32_t*>(&h2);
+                        pk.w = *reinterpret_cast<uint32_t*>(&h3);
+                        *reinterpret_cast<uint4*>(p.D + (d_base + row) * p.N + col) = pk;
                     }
                 }
             }
