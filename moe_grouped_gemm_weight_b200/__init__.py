@@ -98,6 +98,8 @@ def lib() -> ctypes.CDLL:
             L.dg_selftest_bounded_wait.argtypes = [P]
             L.dg_make_plan.restype = I
             L.dg_make_plan.argtypes = [I, I, I, I, I, I, ctypes.POINTER(Plan)]
+            L.dg_make_plan_ue8m0.restype = I
+            L.dg_make_plan_ue8m0.argtypes = [I, I, I, I, ctypes.POINTER(Plan)]
             _lib = L
     return _lib
 
@@ -252,6 +254,12 @@ def dg_make_plan(mode: int, rows: int, N: int, K: int, G: int, num_sms: int) -> 
     pl = Plan()
     _check("dg_make_plan", lib().dg_make_plan(int(mode), int(rows), int(N), int(K), int(G), int(num_sms),
                                               ctypes.byref(pl)))
+    return pl.as_dict()
+
+
+def dg_make_plan_ue8m0(M: int, N: int, K: int, num_sms: int) -> dict:
+    pl = Plan()
+    _check("dg_make_plan_ue8m0", lib().dg_make_plan_ue8m0(int(M), int(N), int(K), int(num_sms), ctypes.byref(pl)))
     return pl.as_dict()
 
 

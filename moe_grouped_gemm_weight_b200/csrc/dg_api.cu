@@ -919,6 +919,33 @@ static int ue8m0_split(int tiles, int nkb, int sms) {
     return split >= 2 ? split : 1;
 }
 
+// Launch plan of the block-scaled kernel: 128 x kUeBN tiles, persistent on
+// at most `sms` CTAs, plus the K-split above (with fewer tiles than SMs,
+// every tile is split and the grid is tiles x split).
+static void ue8m0_plan(int M, int N, int K, int sms, dg_plan* pl) {
+    *pl = dg_plan{};
+    pl->block_m = dg::kBM;
+    pl->block_n = dg::kUeBN;
+    pl->stages = dg::kUeStages;
+    pl->m_blocks = cdiv(M, dg::kBM);
+    pl->n_blocks = cdiv(N, dg::kUeBN);
+    pl->tiles = pl->m_blocks * pl->n_blocks;
+    pl->grid = pl->tiles < sms ? pl->tiles : sms;
+    pl->smem_bytes = dg::ue8m0_smem_bytes();
+    pl->split_k = 1;
+    pl->tail_split = ue8m0_split(pl->tiles, K / dg::kBK, sms);
+    if (pl->tail_split > 1 && pl->tiles < sms) pl->grid = pl->tiles * pl->tail_split;
+}
+
+dg_status dg_make_plan_ue8m0(int M, int N, int K, int num_sms, dg_plan* out) {
+    if (!out) return fail(DG_ERR_INVALID_ARG, "null plan pointer");
+    dg_status s = check_sizes(0, M, N, K, 1);
+    if (s != DG_OK) return s;
+    if (num_sms <= 0) return fail(DG_ERR_INVALID_ARG, "num_sms must be positive");
+    ue8m0_plan(M, N, K, num_sms, out);
+    return DG_OK;
+}
+
 dg_status dg_fp8_gemm_nt_ue8m0(uint16_t* D, const uint8_t* A, const float* sa, int sa_stride, const uint8_t* B,
                                const float* sb, int M, int N, int K, void* stream) {
     dg_status s = check_sizes(0, M, N, K, 1);
@@ -942,17 +969,8 @@ dg_status dg_fp8_gemm_nt_ue8m0(uint16_t* D, const uint8_t* A, const float* sa, i
         if (force && force[0] == '0') block_scaled = false;
         if (!block_scaled) return dg_fp8_gemm_nt(D, A, sa, sa_stride, B, sb, M, N, K, stream);
     }
-    dg_plan pl{};
-    pl.block_m = dg::kBM;
-    pl.block_n = dg::kUeBN;
-    pl.stages = dg::kUeStages;
-    pl.m_blocks = cdiv(M, dg::kBM);
-    pl.n_blocks = cdiv(N, dg::kUeBN);
-    pl.tiles = pl.m_blocks * pl.n_blocks;
-    pl.grid = pl.tiles < sms ? pl.tiles : sms;
-    pl.split_k = 1;
-    pl.tail_split = ue8m0_split(pl.tiles, K / dg::kBK, sms);
-    if (pl.tail_split > 1 && pl.tiles < sms) pl.grid = pl.tiles * pl.tail_split;
+    dg_plan pl;
+    ue8m0_plan(M, N, K, sms, &pl);
     CUtensorMap ta, tb, td;
     if ((s = make_operand_map(&ta, A, K, M, 1, dg::kBM, false)) != DG_OK) return s;
     if ((s = make_operand_map(&tb, B, K, N, 1, dg::kUeBN, true)) != DG_OK) return s;

@@ -103,3 +103,64 @@ def test_few_row_split_grows_with_k_until_the_cluster_cap():
     got = [dg.dg_make_plan(0, 64, 128, 128 * nkb, 1, 148)["split_k"] for nkb in (4, 8, 15, 16, 24, 32, 64, 256)]
     assert got == [1, 1, 3, 4, 6, 8, 8, 8]
     assert all(a <= b for a, b in zip(got, got[1:]))
+
+
+@st.composite
+def block_scaled_problems(draw):
+    M = draw(st.one_of(st.integers(0, 256), st.integers(257, 20000)))
+    N = 8 * draw(st.integers(1, 8192))
+    K = 128 * draw(st.integers(1, 256))
+    return M, N, K, draw(st.integers(1, 148))
+
+
+@settings(max_examples=600, deadline=None, suppress_health_check=[HealthCheck.too_slow])
+@given(block_scaled_problems())
+def test_block_scaled_plan_invariants(problem):
+    """The block-scaled kernel: 128 x 256 tiles, persistent on at most one CTA
+    per SM, and a K-split of the partial last wave (of every tile, when there
+    are fewer tiles than SMs) into 2..8 slices of >= 16 K blocks whose
+    partials fit the workspace's one partial per SM."""
+    M, N, K, sms = problem
+    p = dg.dg_make_plan_ue8m0(M, N, K, sms)
+    nkb = K // 128
+    assert (p["block_m"], p["block_n"]) == (128, 256)
+    assert p["m_blocks"] == cdiv(M, 128) and p["n_blocks"] == cdiv(N, 256)
+    assert p["tiles"] == p["m_blocks"] * p["n_blocks"]
+    assert p["stages"] >= 2 and 113 * 1024 < p["smem_bytes"] <= 227 * 1024
+    assert p["swap_ab"] == 0 and p["split_k"] == 1
+    S = p["tail_split"]
+    tiles = p["tiles"]
+    if S == 1:
+        assert p["grid"] == min(tiles, sms)
+        return
+    rest = tiles % sms
+    assert rest > 0 and 2 <= S <= 8 and nkb // S >= 16 and rest * S <= sms
+    if tiles < sms:
+        assert p["grid"] == tiles * S
+        partials = tiles * (S - 1)
+    else:
+        assert p["grid"] == sms
+        partials = rest * (S - 1)
+    assert partials < sms
+
+
+def test_block_scaled_split_follows_the_tail_rule():
+    # 300 x 520: 3 x 3 tiles.  S ~ sqrt(nkb / 1.5) rounded, capped by 8, by
+    # SMs / leftover tiles and by nkb / 16.
+    assert dg.dg_make_plan_ue8m0(300, 520, 6400, 148)["tail_split"] == 3   # nkb 50: 16/17/17
+    assert dg.dg_make_plan_ue8m0(300, 520, 6400, 148)["grid"] == 27
+    assert dg.dg_make_plan_ue8m0(300, 520, 2048, 148)["tail_split"] == 1   # nkb 16: no room
+    assert dg.dg_make_plan_ue8m0(300, 520, 16384, 148)["tail_split"] == 8  # nkb 128: the cap
+    assert dg.dg_make_plan_ue8m0(300, 520, 16384, 20)["tail_split"] == 2   # 9 tiles on 20 SMs
+    # 4096 x 7168: 32 x 28 = 896 tiles, 6 full waves and 8 left over.
+    p = dg.dg_make_plan_ue8m0(4096, 7168, 16384, 148)
+    assert (p["tiles"], p["grid"], p["tail_split"]) == (896, 148, 8)
+    # A whole number of waves needs no split.
+    assert dg.dg_make_plan_ue8m0(128 * 148, 256, 16384, 148)["tail_split"] == 1
+
+
+def test_block_scaled_plan_rejects_what_the_call_rejects():
+    for args in [(64, 512, 1000, 148), (64, 500, 1024, 148), (-1, 512, 1024, 148), (64, 512, 1024, 0)]:
+        with pytest.raises(RuntimeError):
+            dg.dg_make_plan_ue8m0(*args)
+    assert dg.dg_make_plan_ue8m0(0, 512, 1024, 148)["tiles"] == 0
