@@ -115,6 +115,60 @@ def _ptr(t) -> int:
     return 0 if t is None else int(t.data_ptr())
 
 
+def _cdiv(a: int, b: int) -> int:
+    return -(-a // b)
+
+
+def _sa_need(kblocks: int, sa_stride: int, rows: int) -> int:
+    """Elements of a transposed scale array sa[kb*sa_stride + m] that the
+    library touches for kb < kblocks, m < rows."""
+    return 0 if kblocks <= 0 or rows <= 0 else (kblocks - 1) * int(sa_stride) + rows
+
+
+def _check_dim(func: str, what: str, got: int, want: int) -> None:
+    if got != want:
+        raise DGError(func, DG_ERR_INVALID_ARG, f"{what} is {got}, expected {want}")
+
+
+def _check_args(func: str, *specs) -> None:
+    """Check the tensor arguments before their pointers cross the C boundary.
+
+    Each spec is (name, tensor, element bytes, elements the call touches).  The
+    C ABI takes plain device pointers and cannot see extents, so a tensor that
+    is too short, strided, of another element type, or not on the current CUDA
+    device would be read or written outside its memory by the kernels.  Such a
+    call raises DGError (DG_ERR_INVALID_ARG) here and launches nothing.  None
+    passes through: the library itself reports a null pointer."""
+    given = [sp for sp in specs if sp[1] is not None]
+    for name, t, esize, need in given:
+        if t.element_size() != esize:
+            raise DGError(func, DG_ERR_INVALID_ARG,
+                          f"{name} has {t.element_size()}-byte elements, the call takes {esize}-byte ones")
+        if not t.is_contiguous():
+            raise DGError(func, DG_ERR_INVALID_ARG, f"{name} is not contiguous")
+        if t.numel() < need:
+            raise DGError(func, DG_ERR_INVALID_ARG, f"{name} holds {t.numel()} elements, the call touches {need}")
+    for name, t, _, _ in given:
+        if t.device.type != "cuda":
+            raise DGError(func, DG_ERR_INVALID_ARG, f"{name} is not on a CUDA device ({t.device})")
+    if given:
+        import torch
+        cur = torch.cuda.current_device()
+        for name, t, _, _ in given:
+            if t.device.index != cur:
+                raise DGError(func, DG_ERR_INVALID_ARG, f"{name} is on {t.device}, the current device is cuda:{cur}")
+
+
+def _check_dense(func: str, D, A, sa, sa_stride, B, sb, M: int, N: int, K: int, b_k: int) -> None:
+    """Arguments of a dense call: D [M][N] bf16, A with M*K codes, sa
+    transposed per 1x128, B with N*K codes (its K extent b_k), sb
+    [ceil(N/128)][K/128]."""
+    _check_dim(func, "K of B", b_k, K)
+    nkb = _cdiv(K, 128)
+    _check_args(func, ("D", D, 2, M * N), ("A", A, 1, M * K), ("sa", sa, 4, _sa_need(nkb, sa_stride, M)),
+                ("B", B, 1, N * K), ("sb", sb, 4, _cdiv(N, 128) * nkb))
+
+
 def _stream(stream) -> int:
     if stream is None:
         import torch
@@ -126,6 +180,7 @@ def dg_fp8_gemm_nt(D, A, sa, sa_stride: int, B, sb, stream=None) -> None:
     """Dense D[M,N] = scaled A[M,K] . B[N,K]^T (sizes taken from A and B)."""
     M, K = A.shape[-2], A.shape[-1]
     N = B.shape[-2]
+    _check_dense("dg_fp8_gemm_nt", D, A, sa, sa_stride, B, sb, M, N, K, B.shape[-1])
     _check("dg_fp8_gemm_nt", lib().dg_fp8_gemm_nt(_ptr(D), _ptr(A), _ptr(sa), int(sa_stride), _ptr(B), _ptr(sb),
                                                   M, N, K, _stream(stream)))
 
@@ -134,6 +189,7 @@ def dg_fp8_gemm_nn(D, A, sa, sa_stride: int, B, sb, stream=None) -> None:
     """D[M,N] = scaled A . B^T with A [M,K] and B stored [K,N]."""
     M, K = A.shape[-2], A.shape[-1]
     N = B.shape[-1]
+    _check_dense("dg_fp8_gemm_nn", D, A, sa, sa_stride, B, sb, M, N, K, B.shape[-2])
     _check("dg_fp8_gemm_nn", lib().dg_fp8_gemm_nn(_ptr(D), _ptr(A), _ptr(sa), int(sa_stride), _ptr(B), _ptr(sb),
                                                   M, N, K, _stream(stream)))
 
@@ -142,6 +198,7 @@ def dg_fp8_gemm_tn(D, A, sa, sa_stride: int, B, sb, stream=None) -> None:
     """D[M,N] = scaled A . B^T with A stored [K,M] and B stored [K,N]."""
     K, M = A.shape[-2], A.shape[-1]
     N = B.shape[-1]
+    _check_dense("dg_fp8_gemm_tn", D, A, sa, sa_stride, B, sb, M, N, K, B.shape[-2])
     _check("dg_fp8_gemm_tn", lib().dg_fp8_gemm_tn(_ptr(D), _ptr(A), _ptr(sa), int(sa_stride), _ptr(B), _ptr(sb),
                                                   M, N, K, _stream(stream)))
 
@@ -150,6 +207,7 @@ def dg_fp8_gemm_tt(D, A, sa, sa_stride: int, B, sb, stream=None) -> None:
     """D[M,N] = scaled A . B^T with A stored [K,M] and B [N,K]."""
     K, M = A.shape[-2], A.shape[-1]
     N = B.shape[-2]
+    _check_dense("dg_fp8_gemm_tt", D, A, sa, sa_stride, B, sb, M, N, K, B.shape[-1])
     _check("dg_fp8_gemm_tt", lib().dg_fp8_gemm_tt(_ptr(D), _ptr(A), _ptr(sa), int(sa_stride), _ptr(B), _ptr(sb),
                                                   M, N, K, _stream(stream)))
 
@@ -160,6 +218,11 @@ def dg_k_grouped_fp8_gemm_tn(D, A, sa, sa_stride: int, B, sb, k_offsets, stream=
     K, M = A.shape[-2], A.shape[-1]
     N = B.shape[-1]
     G = k_offsets.numel() - 1
+    func = "dg_k_grouped_fp8_gemm_tn"
+    _check_dim(func, "K of B", B.shape[-2], K)
+    nkb = _cdiv(K, 128)
+    _check_args(func, ("D", D, 2, max(G, 0) * M * N), ("A", A, 1, M * K), ("sa", sa, 4, _sa_need(nkb, sa_stride, M)),
+                ("B", B, 1, N * K), ("sb", sb, 4, _cdiv(N, 128) * nkb), ("k_offsets", k_offsets, 4, G + 1))
     _check("dg_k_grouped_fp8_gemm_tn",
            lib().dg_k_grouped_fp8_gemm_tn(_ptr(D), _ptr(A), _ptr(sa), int(sa_stride), _ptr(B), _ptr(sb),
                                           _ptr(k_offsets), G, M, N, K, _stream(stream)))
@@ -169,6 +232,7 @@ def dg_fp8_gemm_nt_ue8m0(D, A, sa, sa_stride: int, B, sb, stream=None) -> None:
     """dg_fp8_gemm_nt for power-of-two sa / sb, scaled inside the tensor core."""
     M, K = A.shape[-2], A.shape[-1]
     N = B.shape[-2]
+    _check_dense("dg_fp8_gemm_nt_ue8m0", D, A, sa, sa_stride, B, sb, M, N, K, B.shape[-1])
     _check("dg_fp8_gemm_nt_ue8m0", lib().dg_fp8_gemm_nt_ue8m0(_ptr(D), _ptr(A), _ptr(sa), int(sa_stride), _ptr(B),
                                                             _ptr(sb), M, N, K, _stream(stream)))
 
@@ -179,6 +243,7 @@ def dg_fp8_gemm_nt_noalloc(D, A, sa, sa_stride: int, B, sb, stream=None) -> None
     the GPU race.  Make the first call on each device before any stream capture."""
     M, K = A.shape[-2], A.shape[-1]
     N = B.shape[-2]
+    _check_dense("dg_fp8_gemm_nt_noalloc", D, A, sa, sa_stride, B, sb, M, N, K, B.shape[-1])
     _check("dg_fp8_gemm_nt_noalloc",
            lib().dg_fp8_gemm_nt_noalloc(_ptr(D), _ptr(A), _ptr(sa), int(sa_stride), _ptr(B), _ptr(sb),
                                         M, N, K, _stream(stream)))
@@ -187,6 +252,8 @@ def dg_fp8_gemm_nt_noalloc(D, A, sa, sa_stride: int, B, sb, stream=None) -> None
 def dg_to_fp8_1x128(Q, sa, sa_stride: int, X, stream=None) -> None:
     """Activation cast: bf16 X [M,K] -> e4m3 Q [M,K] (uint8) and sa[kb*sa_stride + m]."""
     M, K = X.shape[-2], X.shape[-1]
+    _check_args("dg_to_fp8_1x128", ("Q", Q, 1, M * K), ("sa", sa, 4, _sa_need(_cdiv(K, 128), sa_stride, M)),
+                ("X", X, 2, M * K))
     _check("dg_to_fp8_1x128", lib().dg_to_fp8_1x128(_ptr(Q), _ptr(sa), int(sa_stride), _ptr(X), M, K,
                                                     _stream(stream)))
 
@@ -194,13 +261,21 @@ def dg_to_fp8_1x128(Q, sa, sa_stride: int, X, stream=None) -> None:
 def dg_to_fp8_128x128(Q, sb, W, stream=None) -> None:
     """Weight cast: bf16 W [N,K] -> e4m3 Q [N,K] (uint8) and sb [ceil(N/128), K/128]."""
     N, K = W.shape[-2], W.shape[-1]
+    _check_args("dg_to_fp8_128x128", ("Q", Q, 1, N * K), ("sb", sb, 4, _cdiv(N, 128) * _cdiv(K, 128)),
+                ("W", W, 2, N * K))
     _check("dg_to_fp8_128x128", lib().dg_to_fp8_128x128(_ptr(Q), _ptr(sb), _ptr(W), N, K, _stream(stream)))
 
 
 def dg_grouped_contiguous_nt(D, A, sa, sa_stride: int, B, sb, m_indices, stream=None) -> None:
     """Contiguous-layout grouped GEMM; B is [G,N,K], m_indices int32 [M_total]."""
     M, K = A.shape[-2], A.shape[-1]
+    func = "dg_grouped_contiguous_nt"
+    _check_dim(func, "rank of B", B.dim(), 3)
     G, N = B.shape[0], B.shape[1]
+    _check_dim(func, "K of B", B.shape[2], K)
+    nkb = _cdiv(K, 128)
+    _check_args(func, ("D", D, 2, M * N), ("A", A, 1, M * K), ("sa", sa, 4, _sa_need(nkb, sa_stride, M)),
+                ("B", B, 1, G * N * K), ("sb", sb, 4, G * _cdiv(N, 128) * nkb), ("m_indices", m_indices, 4, M))
     _check("dg_grouped_contiguous_nt",
            lib().dg_grouped_contiguous_nt(_ptr(D), _ptr(A), _ptr(sa), int(sa_stride), _ptr(B), _ptr(sb),
                                           _ptr(m_indices), M, N, K, G, _stream(stream)))
@@ -208,8 +283,17 @@ def dg_grouped_contiguous_nt(D, A, sa, sa_stride: int, B, sb, m_indices, stream=
 
 def dg_grouped_masked_nt(D, A, sa, sa_stride: int, B, sb, masked_m, expected_m: int = 0, stream=None) -> None:
     """Masked-layout grouped GEMM; A is [G,M_max,K], masked_m int32 [G] on the device."""
+    func = "dg_grouped_masked_nt"
+    _check_dim(func, "rank of A", A.dim(), 3)
+    _check_dim(func, "rank of B", B.dim(), 3)
     G, Mmax, K = A.shape
     N = B.shape[1]
+    _check_dim(func, "group count of B", B.shape[0], G)
+    _check_dim(func, "K of B", B.shape[2], K)
+    nkb = _cdiv(K, 128)
+    _check_args(func, ("D", D, 2, G * Mmax * N), ("A", A, 1, G * Mmax * K),
+                ("sa", sa, 4, _sa_need(G * nkb, sa_stride, Mmax)), ("B", B, 1, G * N * K),
+                ("sb", sb, 4, G * _cdiv(N, 128) * nkb), ("masked_m", masked_m, 4, G))
     _check("dg_grouped_masked_nt",
            lib().dg_grouped_masked_nt(_ptr(D), _ptr(A), _ptr(sa), int(sa_stride), _ptr(B), _ptr(sb),
                                       _ptr(masked_m), G, Mmax, N, K, int(expected_m), _stream(stream)))
