@@ -440,6 +440,20 @@ dg_status launch_one(const dg::Params& p, const CUtensorMap& ta, const CUtensorM
     if (dev >= 0 && dev < kMaxDevices && !attr_set[dev].load()) {
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
             return fail(DG_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(cudaGetLastError()));
+        using C = dg::Cfg<BN>;
+        if (C::kSplitRegs) {
+            // The setmaxnreg split draws on the registers the CTA is launched
+            // with (its threads x the compiled register count); a build whose
+            // count cannot cover it would wait forever in setmaxnreg, so it is
+            // refused here, before any launch.
+            constexpr int need = 128 * C::kRegsLow + 128 * C::kEpiWGs * C::kRegsHigh;
+            cudaFuncAttributes fa{};
+            if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess)
+                return fail(DG_ERR_CUDA, "cudaFuncGetAttributes: %s", cudaGetErrorString(cudaGetLastError()));
+            if (fa.numRegs * C::kThreadsC < need)
+                return fail(DG_ERR_UNSUPPORTED, "GEMM kernel (BN=%d) compiled with %d registers per thread x %d "
+                            "threads, its register split needs %d", BN, fa.numRegs, C::kThreadsC, need);
+        }
         attr_set[dev].store(1);
     }
     cudaLaunchConfig_t cfg = {};
