@@ -48,7 +48,12 @@
  *             CUDA graph.
  *  Errors     Bad arguments are reported synchronously as a dg_status and
  *             nothing is launched (dg_last_error_message() says why).  A
- *             launch failure returns DG_ERR_CUDA.  Bad DEVICE-side data
+ *             launch failure returns DG_ERR_CUDA.  DG_ERR_UNSUPPORTED also
+ *             reports a library build whose kernel cannot run as compiled:
+ *             before a kernel's first launch the host checks that its
+ *             compiled register count covers the kernel's register split
+ *             (threads x registers per thread), which would otherwise wait
+ *             forever on the device.  Bad DEVICE-side data
  *             (m_indices outside [-1,G), masked_m outside [0,M_max]) cannot be
  *             seen by the host: the kernel skips the offending rows/groups
  *             (masked_m is clamped) and sets a bit in the device error word,
