@@ -93,6 +93,7 @@ def test_ue8m0_k_split(dgm, sms):
     # all nine tiles are split into 3 K slices (27 CTAs); on 7 SMs the two
     # tiles after one full wave are, on 4 SMs the one tile after two waves.
     c = wl.dense_case(300, 520, 6144, seed=11, stress=True)
+    assert dgm.dg_make_plan_ue8m0(300, 520, 6144, sms)["tail_split"] == 3
     dgm.dg_set_num_sms(sms)
     try:
         got = _run(dgm, c)
@@ -111,6 +112,7 @@ def test_ue8m0_uneven_k_split(dgm):
     # K blocks 16 and 33, so their groups of four scale bytes start off the
     # multiples of four.
     c = wl.dense_case(300, 520, 6400, seed=23, stress=True)
+    assert dgm.dg_make_plan_ue8m0(300, 520, 6400, dgm.dg_get_num_sms())["tail_split"] == 3
     got = _run(dgm, c)
     again = _run(dgm, c)
     assert dgm.dg_get_device_error() == 0
@@ -125,6 +127,7 @@ def test_ue8m0_odd_k_blocks_over_many_work_items(dgm, sms):
     # turn -- alternate K blocks, counted over the CTA's work items -- falls
     # on the other warp at every new tile.
     c = wl.dense_case(513, 1032, 640, seed=17, stress=True)
+    assert dgm.dg_make_plan_ue8m0(513, 1032, 640, sms)["tail_split"] == 1
     dgm.dg_set_num_sms(sms)
     try:
         got = _run(dgm, c)
