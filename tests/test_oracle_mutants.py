@@ -35,6 +35,15 @@ MUTANTS = {
     "cast_no_saturation": ("if (a >= 448.0) return sign | 0x7E;", "if (a >= 1e30) return sign | 0x7E;"),
     "cast_half_tile_amax": ("for (int k = c0; k < c0 + 128; ++k) amax = fmaxf",
                             "for (int k = c0; k < c0 + 64; ++k) amax = fmaxf"),
+    "e4m3_subnormal_scale": ("v = ldexp((double)m, -9);", "v = ldexp((double)m, -10);"),
+    "bf16_ties_away": ("r = (fmod(fl, 2.0) == 0.0) ? fl : fl + 1.0;", "r = fl + 1.0;"),
+    "bf16_no_subnormal_spacing": ("if (q < -133) q = -133;", "if (q < -126) q = -126;"),
+    "masked_sa_ignores_group": ("const float* sa_m = sa + (int64_t)g * nkb * sa_stride + m;",
+                                "const float* sa_m = sa + m;"),
+    "masked_b_ignores_group": ("B + (int64_t)g * N * K, sb + (int64_t)g * nbn * nkb, N, K,\n                 D + flat * N",
+                               "B, sb, N, K,\n                 D + flat * N"),
+    "cast_subnormal_scale": ("return sign | (uint8_t)(v / ldexp(1.0, -9));", "return sign | (uint8_t)(v / ldexp(1.0, -10));"),
+    "cast_exponent_bias": ("return sign | (uint8_t)(((E2 + 7) << 3) | mant);", "return sign | (uint8_t)(((E2 + 8) << 3) | mant);"),
     "cast_sa_not_transposed": ("cast_tile(X, K, m, m + 1, kb * 128, Q, sa + (int64_t)kb * sa_stride + m);",
                                "cast_tile(X, K, m, m + 1, kb * 128, Q, sa + (int64_t)m * nkb + kb);"),
 }
