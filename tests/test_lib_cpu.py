@@ -4,6 +4,7 @@ rules, and bad arguments are rejected synchronously before any CUDA call."""
 import ctypes
 import os
 import re
+import subprocess
 
 import pytest
 
@@ -206,3 +207,47 @@ def test_pdl_switch_defaults_to_the_environment(monkeypatch):
         assert dg.dg_get_pdl() is False
     finally:
         dg.dg_set_pdl(None)
+
+
+C_CLIENT = r"""
+#include <stdio.h>
+#include <string.h>
+#include "dg.h"
+
+int main(void) {
+    dg_plan p;
+    dg_status s = dg_make_plan(0, 4096, 7168, 16384, 1, 148, &p);
+    if (s != DG_OK) return 1;
+    printf("plan %d %d %d %d %d\n", p.block_m, p.block_n, p.tiles, p.grid, p.tail_split);
+    s = dg_make_plan_ue8m0(4096, 7168, 16384, 148, &p);
+    if (s != DG_OK) return 2;
+    printf("ue8m0 %d %d %d\n", p.block_n, p.tiles, p.tail_split);
+    printf("align %d %d\n", dg_get_m_alignment_for_contiguous_layout(), dg_get_tma_aligned_size(65, 4));
+    s = dg_make_plan(0, 64, 2112, 100, 1, 148, &p);
+    printf("bad %d %s|%s\n", (int)s, dg_status_string(s), strstr(dg_last_error_message(), "K=100") ? "K" : "?");
+    /* a GEMM call with a null output is refused before any device work */
+    s = dg_fp8_gemm_nt(NULL, NULL, NULL, 64, NULL, NULL, 64, 64, 128, NULL);
+    printf("null %d\n", (int)s);
+    return 0;
+}
+"""
+
+
+def test_header_compiles_as_c99_and_links(tmp_path):
+    """include/dg.h is a C ABI: a plain C99 client (-pedantic -Werror) compiles
+    against it, links libdg.so and calls the host-only functions."""
+    src, exe = tmp_path / "client.c", tmp_path / "client"
+    src.write_text(C_CLIENT)
+    libdir = os.path.dirname(dg.LIB_PATH)
+    cmd = ["gcc", "-std=c99", "-pedantic", "-Wall", "-Wextra", "-Werror", "-I", os.path.join(ROOT, "include"),
+           str(src), "-o", str(exe), "-L", libdir, "-ldg", f"-Wl,-rpath,{libdir}"]
+    r = subprocess.run(cmd, capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    r = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert r.returncode == 0, (r.returncode, r.stdout, r.stderr)
+    lines = dict(l.split(" ", 1) for l in r.stdout.strip().splitlines())
+    assert lines["plan"].split()[:2] == ["128", "256"]
+    assert lines["ue8m0"] == "256 896 8"
+    assert lines["align"] == "128 68"
+    assert lines["bad"] == f"{dg.DG_ERR_UNSUPPORTED} {dg.dg_status_string(dg.DG_ERR_UNSUPPORTED)}|K"
+    assert lines["null"] == str(dg.DG_ERR_INVALID_ARG)
