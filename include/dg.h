@@ -308,9 +308,10 @@ DG_API const char* dg_status_string(dg_status s);
 DG_API const char* dg_last_error_message(void);
 
 /*
- * Launch plan (host only, no GPU needed): what a call with these sizes would
- * launch.  mode: 0 dense, 1 contiguous, 2 masked.  rows = M (dense), M_total
- * (contiguous) or M_max (masked).  Returns DG_ERR_INVALID_ARG for bad sizes.
+ * Launch plan (host only, no GPU needed; no counterpart on the pages): what a
+ * call with these sizes would launch.  mode: 0 dense, 1 contiguous, 2
+ * masked.  rows = M (dense), M_total (contiguous) or M_max (masked).
+ * Returns DG_ERR_INVALID_ARG for bad sizes.
  */
 typedef struct dg_plan {
     int block_m;      /* output rows per tile                                    */
@@ -330,12 +331,13 @@ typedef struct dg_plan {
 DG_API dg_status dg_make_plan(int mode, int rows, int N, int K, int G, int num_sms, dg_plan* out);
 
 /*
- * Launch plan (host only, no GPU needed) of the block-scaled kernel that
- * dg_fp8_gemm_nt_ue8m0 runs when it takes that kernel (M > 256, or
- * DG_FORCE_BLOCK_SCALED=1): 128 x 256 tiles, grid <= num_sms, and
- * tail_split > 1 when the tiles of the last partial wave (all tiles, when
- * there are fewer than num_sms; the grid is then tiles x tail_split) are
- * split along K.  swap_ab is 0 and split_k 1.  M == 0 gives zero tiles.
+ * Launch plan (host only, no GPU needed; no counterpart on the pages) of the
+ * block-scaled kernel that dg_fp8_gemm_nt_ue8m0 runs when it takes that
+ * kernel (M > 256, or DG_FORCE_BLOCK_SCALED=1): 128 x 256 tiles, grid <=
+ * num_sms, and tail_split > 1 when the tiles of the last partial wave (all
+ * tiles, when there are fewer than num_sms; the grid is then tiles x
+ * tail_split) are split along K.  swap_ab is 0 and split_k 1.  M == 0 gives
+ * zero tiles.
  * Returns DG_ERR_INVALID_ARG / DG_ERR_UNSUPPORTED for the sizes
  * dg_fp8_gemm_nt_ue8m0 rejects, or for num_sms <= 0 or a null `out`.
  */
