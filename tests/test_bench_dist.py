@@ -70,3 +70,42 @@ def test_reference_arm_json_line_on_rank_zero():
     assert line["impl"] == "reference" and line["unit"] == "TFLOP/s" and line["value"] > 0
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] == 2
     assert line["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def _dying_worker(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world),
+                      LOCAL_RANK=str(rank))
+    sys.path.insert(0, ROOT)
+    import time
+    import bench
+    bench.dist_init(world, "gloo")
+    bench.barrier(world)
+    if rank == 1:
+        os._exit(3)  # a rank that dies between steps, without leaving the group
+    time.sleep(1.0)
+    t0 = time.monotonic()
+    try:
+        bench.max_over_ranks(1.0, world, "cpu")
+        q.put((rank, "completed", time.monotonic() - t0))
+    except Exception as e:  # the collective must end with an error, not wait
+        q.put((rank, type(e).__name__, time.monotonic() - t0))
+    os._exit(0)
+
+
+def test_a_dead_rank_ends_the_next_collective_with_an_error():
+    """Failure detection on the host: rank 1 dies between steps; rank 0's next
+    timing all-reduce fails with an error within the process group's timeout
+    instead of waiting for ever."""
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_dying_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=200)
+    assert procs[1].exitcode == 3
+    assert procs[0].exitcode == 0, "rank 0 did not come back from its collective"
+    rank, outcome, waited = q.get(timeout=10)
+    assert rank == 0 and outcome != "completed", outcome
+    assert waited < 130
