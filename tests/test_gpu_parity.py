@@ -77,8 +77,11 @@ def oracle_dense(c: wl.Case, rows=None):
 
 # --------------------------------------------------------------- dense -----
 
+# ... plus the narrowest output the layout allows (N = 8: one 16-byte row of
+# D) on the few-row kernel and on the 128-row tile kernel.
 DENSE_SMALL = [(1, 64, 128), (64, 64, 256), (127, 200, 384), (128, 128, 128), (129, 136, 512),
-               (300, 264, 1024), (256, 520, 640), (513, 1032, 256), (64, 2112, 7168)]
+               (300, 264, 1024), (256, 520, 640), (513, 1032, 256), (64, 2112, 7168), (1, 8, 128),
+               (300, 8, 256)]
 
 
 @pytest.mark.parametrize("M,N,K", DENSE_SMALL)
@@ -197,8 +200,11 @@ def check_masked_untouched(got, masked_m):
         assert np.all(got[g, mm:] == SENTINEL), f"group {g}: rows past masked_m were written"
 
 
+# The last two: every group empty on the 128-row tile kernel (M_max > 256;
+# D must stay untouched), and N = 8 on the few-row kernel.
 @pytest.mark.parametrize("G,Mmax,N,K,mm", [(3, 200, 136, 256, [0, 200, 65]), (1, 5, 64, 128, [5]),
-                                           (5, 130, 264, 384, [129, 1, 130, 0, 128])])
+                                           (5, 130, 264, 384, [129, 1, 130, 0, 128]),
+                                           (2, 300, 136, 256, [0, 0]), (2, 40, 8, 128, [40, 0])])
 def test_masked_small_full(dgm, G, Mmax, N, K, mm):
     c = wl.masked_case(G, Mmax, N, K, masked_m=mm, seed=G + Mmax)
     got = run_masked(dgm, c)
@@ -263,7 +269,7 @@ def test_masked_under_cuda_graph_follows_device_counts(dgm):
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g, stream=s):
         dgm.dg_grouped_masked_nt(D, cg.A, cg.sa, cg.sa_stride, cg.B, cg.sb, cg.masked_m, 128)
-    for counts in ([1, 2, 3, 4], [256, 0, 0, 200]):
+    for counts in ([1, 2, 3, 4], [256, 0, 0, 200], [0, 0, 0, 0]):
         D.view(torch.int16).fill_(SENTINEL)
         cg.masked_m.copy_(torch.tensor(counts, dtype=torch.int32))
         g.replay()
