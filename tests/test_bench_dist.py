@@ -89,6 +89,10 @@ def _dying_worker(rank, world, port, q):
         q.put((rank, "completed", time.monotonic() - t0))
     except Exception as e:  # the collective must end with an error, not wait
         q.put((rank, type(e).__name__, time.monotonic() - t0))
+    # Flush the queue's feeder thread before leaving without the process
+    # group's normal shutdown (which would wait on the dead peer).
+    q.close()
+    q.join_thread()
     os._exit(0)
 
 
