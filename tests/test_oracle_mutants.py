@@ -7,6 +7,7 @@ run against it in a subprocess and must fail.  The real oracle is untouched.
 import os
 import subprocess
 import sys
+from concurrent.futures import ThreadPoolExecutor
 
 import pytest
 
@@ -49,18 +50,38 @@ MUTANTS = {
 }
 
 
-@pytest.mark.parametrize("name", sorted(MUTANTS))
-def test_pins_reject_mutant(name, tmp_path):
+def _run_mutant(name: str, workdir: str):
+    """Compile mutant `name` and run the pin suite against it; returns
+    (pin suite exit code, tail of its output)."""
     old, new = MUTANTS[name]
     src = open(SRC).read()
-    assert src.count(old) == 1, f"mutation site for {name} not found exactly once"
-    mut = tmp_path / "mutant.c"
-    mut.write_text(src.replace(old, new))
-    so = tmp_path / "libmutant.so"
+    if src.count(old) != 1:
+        return None, f"mutation site for {name} not found exactly once"
+    mut = os.path.join(workdir, f"{name}.c")
+    so = os.path.join(workdir, f"lib{name}.so")
+    with open(mut, "w") as f:
+        f.write(src.replace(old, new))
     subprocess.run(["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c11", "-ffp-contract=off",
-                    str(mut), "-o", str(so), "-lm"], check=True)
-    env = dict(os.environ, DG_ORACLE_SO=str(so), OMP_NUM_THREADS="2")
+                    mut, "-o", so, "-lm"], check=True)
+    env = dict(os.environ, DG_ORACLE_SO=so, OMP_NUM_THREADS="2")
     r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
                         os.path.join(ROOT, "tests", "test_oracle_pins.py")],
-                       cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
-    assert r.returncode != 0, f"mutant {name} passed every pin:\n{r.stdout[-2000:]}"
+                       cwd=ROOT, env=env, capture_output=True, text=True, timeout=900)
+    return r.returncode, r.stdout[-2000:]
+
+
+@pytest.fixture(scope="module")
+def mutant_results(tmp_path_factory):
+    """Every mutant's pin-suite run, four at a time (each run is its own
+    process with two OpenMP threads)."""
+    workdir = str(tmp_path_factory.mktemp("mutants"))
+    with ThreadPoolExecutor(max_workers=4) as ex:
+        futs = {n: ex.submit(_run_mutant, n, workdir) for n in sorted(MUTANTS)}
+        return {n: f.result() for n, f in futs.items()}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_pins_reject_mutant(name, mutant_results):
+    code, out = mutant_results[name]
+    assert code is not None, out
+    assert code != 0, f"mutant {name} passed every pin:\n{out}"
